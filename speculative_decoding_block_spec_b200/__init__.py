@@ -1,0 +1,259 @@
+"""specv — batched verification and acceptance of block-diffusion speculative
+drafts on NVIDIA B200 (sm_100a).
+
+This module is a thin ctypes binding over libspecv.so, whose C ABI is
+declared in include/specv.h. It only marshals torch CUDA tensors into
+pointers and sizes; every step of the computation runs in the library's CUDA
+kernels. There is no CPU fallback: if the library is not built, or a tensor
+is not on a CUDA device, the call raises.
+
+Entry points (same names as the C ABI):
+  softmax_T(logits, T, probs=False)             temperature softmax statistics
+  spec_verify_block(target, draft, tokens, u, g, T, ...)
+  spec_verify_mixture(target, draft, mix_w, tokens, u, g, T, ...)
+  dvl_allocate_pack(scores, budget, dense_target=None, packed_target=None)
+Workspaces: Workspace(nbytes, device), with verify/softmax/dvl size helpers.
+"""
+import ctypes
+import os
+
+import torch
+
+__all__ = ["SpecError", "Workspace", "lib", "softmax_T", "spec_softmax_T", "spec_verify_block",
+           "spec_verify_mixture", "spec_verify_window_stats", "spec_verify_accept", "dvl_allocate_pack", "verify_workspace_size", "softmax_workspace_size",
+           "dvl_workspace_size", "LIB_PATH", "EXPORTS", "DEV_TOKEN_RANGE", "DEV_NONFINITE", "DEV_VERIFY_LEN",
+           "DEV_SCORES", "DEV_TIMEOUT"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libspecv.so")
+
+DEV_TOKEN_RANGE, DEV_NONFINITE, DEV_VERIFY_LEN, DEV_SCORES, DEV_TIMEOUT = 1, 2, 4, 8, 16
+_F32, _BF16 = 0, 1
+
+_P, _I, _I64, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+_SIGS = {
+    "spec_status_string": ([_I], ctypes.c_char_p),
+    "spec_softmax_workspace_size": ([_I64], _SZ),
+    "spec_verify_workspace_size": ([_I, _I, _I, _I64], _SZ),
+    "spec_dvl_workspace_size": ([_I], _SZ),
+    "spec_workspace_init": ([_P, _SZ, _P], _I),
+    "spec_softmax_T": ([_P, _I, _I64, _I64, _I64, _F, _P, _P, _P, _P, _SZ, _P], _I),
+    "spec_verify_block": ([_P, _P, _P, _I, _P, _P, _P, _P, _I, _I, _I64, _F, _P, _P, _P, _SZ, _P], _I),
+    "spec_verify_mixture": ([_P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _I, _I, _I64, _F, _P, _P, _P, _SZ, _P], _I),
+    "spec_verify_window_stats": ([_P, _P, _P, _I, _I, _P, _I, _I, _I64, _F, _P, _SZ, _P], _I),
+    "spec_verify_accept": ([_P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _I, _I, _I64, _F, _P, _P, _P, _SZ, _P], _I),
+    "dvl_allocate_pack": ([_P, _I, _I, _I, _P, _P, _P, _P, _P, _I, _I64, _P, _SZ, _P], _I),
+}
+EXPORTS = tuple(_SIGS)
+
+_lib = None
+
+
+class SpecError(RuntimeError):
+    """A specv call was rejected (negative spec_status)."""
+
+    def __init__(self, fn, status):
+        super().__init__("%s: %s" % (fn, lib().spec_status_string(status).decode()))
+        self.status = status
+
+
+def lib():
+    """Load libspecv.so (built in-tree by `python -m speculative_decoding_block_spec_b200.build`)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libspecv.so is not built (%s); run "
+                               "`python -m speculative_decoding_block_spec_b200.build`" % LIB_PATH)
+        h = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            fn = getattr(h, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = h
+    return _lib
+
+
+def _call(name, *args):
+    st = getattr(lib(), name)(*args)
+    if st != 0:
+        raise SpecError(name, st)
+
+
+def softmax_workspace_size(rows):
+    return int(lib().spec_softmax_workspace_size(rows))
+
+
+def verify_workspace_size(B, L, K=1, V=151936):
+    return int(lib().spec_verify_workspace_size(B, L, K, V))
+
+
+def dvl_workspace_size(B):
+    return int(lib().spec_dvl_workspace_size(B))
+
+
+class Workspace:
+    """A caller-owned, fixed-address device workspace, zeroed once at creation."""
+
+    def __init__(self, nbytes, device=None):
+        if nbytes <= 0:
+            raise ValueError("workspace size must be positive (shape outside the supported limits?)")
+        self.buf = torch.empty(int(nbytes), dtype=torch.uint8, device=device or "cuda")
+        self.init()
+
+    @property
+    def nbytes(self):
+        return self.buf.numel()
+
+    def ptr(self):
+        return self.buf.data_ptr()
+
+    def init(self):
+        _call("spec_workspace_init", self.ptr(), self.nbytes, _stream(self.buf))
+
+    def status(self):
+        """Sticky device status (OR of DEV_* flags); synchronises the current stream."""
+        return int(self.buf[:4].view(torch.int32).item())
+
+
+def _stream(t):
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _dtype_code(t):
+    if t.dtype == torch.float32:
+        return _F32
+    if t.dtype == torch.bfloat16:
+        return _BF16
+    raise TypeError("logits must be float32 or bfloat16, got %s" % t.dtype)
+
+
+def _dev(t, name, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    return t.data_ptr()
+
+
+def _opt(t, name, dtype):
+    return None if t is None else _dev(t, name, dtype)
+
+
+def spec_softmax_T(logits, T, row_max, row_lse, probs=None, workspace=None):
+    """C-ABI spec_softmax_T on preallocated outputs. logits [rows, V] (row stride V)."""
+    rows, V = logits.shape
+    ws = workspace or Workspace(softmax_workspace_size(rows), logits.device)
+    _call("spec_softmax_T", _dev(logits, "logits"), _dtype_code(logits), rows, V, V, float(T),
+          _dev(row_max, "row_max", torch.float32), _dev(row_lse, "row_lse", torch.float32),
+          _opt(probs, "probs", torch.float32), ws.ptr(), ws.nbytes, _stream(logits))
+    return ws
+
+
+def softmax_T(logits, T, probs=False, workspace=None):
+    """Temperature softmax of each row of logits [rows, V]: returns (row_max,
+    row_lse) of z = logits / T, plus fp32 probabilities if probs=True."""
+    rows, V = logits.shape
+    rmax = torch.empty(rows, dtype=torch.float32, device=logits.device)
+    rlse = torch.empty_like(rmax)
+    p = torch.empty((rows, V), dtype=torch.float32, device=logits.device) if probs else None
+    spec_softmax_T(logits, T, rmax, rlse, p, workspace)
+    return (rmax, rlse, p) if probs else (rmax, rlse)
+
+
+def _outputs(B, L, device, out):
+    if out is None:
+        return (torch.empty(B, dtype=torch.int32, device=device),
+                torch.empty((B, L + 1), dtype=torch.int32, device=device))
+    return out
+
+
+def spec_verify_block(target, draft, tokens, u, g, T, *, verify_len=None, target_row_off=None, workspace=None,
+                      out=None):
+    """Verify B independently drafted blocks. target [B, L+1, V] (or packed rows
+    [S, V] with target_row_off [B]), draft [B, L, V], tokens [B, L] int32,
+    u [B, L] fp32, g [B, L+1, V] fp32. Returns (accept_len [B], out_tokens [B, L+1])."""
+    B, L = tokens.shape
+    V = draft.shape[-1]
+    ws = workspace or Workspace(verify_workspace_size(B, L, 1, V), draft.device)
+    acc, outt = _outputs(B, L, draft.device, out)
+    if _dtype_code(target) != _dtype_code(draft):
+        raise TypeError("target and draft logits must share a dtype")
+    _call("spec_verify_block", _dev(target, "target"), _opt(target_row_off, "target_row_off", torch.int32),
+          _dev(draft, "draft"), _dtype_code(draft), _dev(tokens, "tokens", torch.int32),
+          _opt(verify_len, "verify_len", torch.int32), _dev(u, "u", torch.float32), _dev(g, "g", torch.float32),
+          B, L, V, float(T), _dev(acc, "accept_len", torch.int32), _dev(outt, "out_tokens", torch.int32),
+          ws.ptr(), ws.nbytes, _stream(draft))
+    return acc, outt
+
+
+def spec_verify_mixture(target, draft, mix_w, tokens, u, g, T, *, verify_len=None, target_row_off=None,
+                        workspace=None, out=None):
+    """Verify B latent-mixture drafts: draft [B, K, L, V], mix_w [B, K] fp32
+    (category probabilities q(z|y)); other arguments as spec_verify_block."""
+    B, L = tokens.shape
+    K, V = draft.shape[1], draft.shape[-1]
+    ws = workspace or Workspace(verify_workspace_size(B, L, K, V), draft.device)
+    acc, outt = _outputs(B, L, draft.device, out)
+    if _dtype_code(target) != _dtype_code(draft):
+        raise TypeError("target and draft logits must share a dtype")
+    _call("spec_verify_mixture", _dev(target, "target"), _opt(target_row_off, "target_row_off", torch.int32),
+          _dev(draft, "draft"), _dev(mix_w, "mix_w", torch.float32), K, _dtype_code(draft),
+          _dev(tokens, "tokens", torch.int32), _opt(verify_len, "verify_len", torch.int32),
+          _dev(u, "u", torch.float32), _dev(g, "g", torch.float32), B, L, V, float(T),
+          _dev(acc, "accept_len", torch.int32), _dev(outt, "out_tokens", torch.int32), ws.ptr(), ws.nbytes,
+          _stream(draft))
+    return acc, outt
+
+
+def spec_verify_window_stats(target, draft, T, workspace, *, K=1, L=None, verify_len=None, target_row_off=None):
+    """Stage 1 of verification: temperature-softmax statistics of the verify
+    window into `workspace` (draft [B, L, V] for K == 1, else [B, K, L, V])."""
+    B = target.shape[0] if target_row_off is None else target_row_off.shape[0]
+    L = draft.shape[-2] if L is None else L
+    V = draft.shape[-1]
+    _call("spec_verify_window_stats", _dev(target, "target"), _opt(target_row_off, "target_row_off", torch.int32),
+          _dev(draft, "draft"), K, _dtype_code(draft), _opt(verify_len, "verify_len", torch.int32), B, L, V,
+          float(T), workspace.ptr(), workspace.nbytes, _stream(draft))
+
+
+def spec_verify_accept(target, draft, tokens, u, g, T, workspace, *, mix_w=None, verify_len=None,
+                       target_row_off=None, out=None):
+    """Stage 2 of verification (after spec_verify_window_stats on the same
+    workspace): accept tests, first rejection and the terminal draw."""
+    B, L = tokens.shape
+    K = 1 if draft.dim() == 3 else draft.shape[1]
+    V = draft.shape[-1]
+    acc, outt = _outputs(B, L, draft.device, out)
+    _call("spec_verify_accept", _dev(target, "target"), _opt(target_row_off, "target_row_off", torch.int32),
+          _dev(draft, "draft"), _opt(mix_w, "mix_w", torch.float32), K, _dtype_code(draft),
+          _dev(tokens, "tokens", torch.int32), _opt(verify_len, "verify_len", torch.int32),
+          _dev(u, "u", torch.float32), _dev(g, "g", torch.float32), B, L, V, float(T),
+          _dev(acc, "accept_len", torch.int32), _dev(outt, "out_tokens", torch.int32), workspace.ptr(),
+          workspace.nbytes, _stream(draft))
+    return acc, outt
+
+
+def dvl_allocate_pack(scores, budget, *, dense_target=None, packed_target=None, workspace=None, out=None):
+    """DVL allocation from survival scores [B, L] fp32 under `budget` slots.
+    Returns (verify_len [B], offsets [B+1], slot_map [budget]) int32; if
+    dense_target [B, L+1, V] and packed_target [budget, V] are given, the
+    selected rows are copied into packed_target."""
+    B, L = scores.shape
+    dev = scores.device
+    ws = workspace or Workspace(dvl_workspace_size(B), dev)
+    if out is None:
+        out = (torch.empty(B, dtype=torch.int32, device=dev), torch.empty(B + 1, dtype=torch.int32, device=dev),
+               torch.empty(max(int(budget), 0), dtype=torch.int32, device=dev))
+    vl, off, sm = out
+    dptr = pptr = None
+    dt, V = 0, 1
+    if dense_target is not None or packed_target is not None:
+        if dense_target is None or packed_target is None:
+            raise ValueError("dense_target and packed_target go together")
+        dt, V = _dtype_code(dense_target), dense_target.shape[-1]
+        dptr, pptr = _dev(dense_target, "dense_target"), _dev(packed_target, "packed_target", dense_target.dtype)
+    _call("dvl_allocate_pack", _dev(scores, "scores", torch.float32), B, L, int(budget),
+          _dev(vl, "verify_len", torch.int32), _dev(off, "offsets", torch.int32),
+          _opt(sm, "slot_map", torch.int32), dptr, pptr, dt, V, ws.ptr(), ws.nbytes, _stream(scores))
+    return vl, off, sm

@@ -1,0 +1,355 @@
+// C ABI of specv (declared in include/specv.h): host-side argument checks,
+// workspace carving and kernel launches. No call allocates, frees or
+// synchronises; every launch is stream-ordered.
+#include <algorithm>
+#include <cmath>
+#include <mutex>
+
+#include "specv.h"
+#include "common.cuh"
+#include "internal.h"
+
+using namespace specv;
+
+namespace {
+
+constexpr size_t kHeader = 256;  // status word + padding
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+bool aligned(const void* p, size_t a) { return reinterpret_cast<uintptr_t>(p) % a == 0; }  // NULL is aligned
+int esize(int dtype) { return dtype == SPEC_F32 ? 4 : 2; }
+bool dtype_ok(int dtype) { return dtype == SPEC_F32 || dtype == SPEC_BF16; }
+
+int map_cuda(cudaError_t e) { return e == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA; }
+
+int sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  static std::mutex mu;
+  static int cache[64] = {0};
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 64 && cache[dev]) return cache[dev];
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) sms = 148;
+  if (dev < 64) cache[dev] = sms;
+  return sms;
+}
+
+// Verify workspace: persistent state first (never overlapped), then scratch
+// that the fused and the two-stage paths share.
+struct VerifyLayout {
+  size_t ctl, req_cnt, tterm, dready, tickets;       // persistent counters and flags
+  size_t tpart, rpart;                               // two-stage scratch
+  size_t dec, tpart_f, xg, part_f;                   // fused scratch
+  size_t total;
+};
+
+VerifyLayout verify_layout(int B, int L, int K, int64_t V) {
+  VerifyLayout l;
+  const size_t b4 = align256(static_cast<size_t>(B) * sizeof(int));
+  l.ctl = kHeader;
+  l.req_cnt = l.ctl + 256;
+  l.tterm = l.req_cnt + b4;
+  l.dready = l.tterm + b4;
+  l.tickets = l.dready + b4;
+  const size_t scratch = l.tickets + b4;
+  const size_t rows = static_cast<size_t>(B) * (K + 1) * L;
+  l.tpart = scratch;
+  l.rpart = l.tpart + align256(static_cast<size_t>(B) * kPMax * sizeof(TermPart));
+  const size_t split_end = l.rpart + align256((static_cast<size_t>(kGMax) + rows) * sizeof(float2));
+  const size_t cpr = static_cast<size_t>(fused_cpr(std::max<int64_t>(V, 1), SPEC_F32));
+  l.dec = scratch;
+  l.tpart_f = l.dec + align256(static_cast<size_t>(B) * sizeof(Decision));
+  l.xg = l.tpart_f + align256(static_cast<size_t>(B) * kFusedPtMax * sizeof(TermPart));
+  l.part_f = l.xg + align256(rows * sizeof(float));
+  const size_t fused_end = l.part_f + align256(rows * cpr * sizeof(float2));
+  l.total = std::max(split_end, fused_end);
+  return l;
+}
+
+bool verify_shape_ok(int B, int L, int K) {
+  return B >= 1 && B <= SPEC_MAX_B && L >= 0 && L <= SPEC_MAX_L && K >= 1 && K <= SPEC_MAX_K;
+}
+
+// Checks shared by the verify entry points. Returns SPEC_OK or a negative status.
+int verify_check(const void* target, const int32_t* row_off, const void* draft, const float* mix_w, int K,
+                 int dtype, const int32_t* tokens, const int32_t* vlen, const float* u, const float* g, int B, int L,
+                 int64_t V, float T, const int32_t* accept_len, const int32_t* out_tokens, const void* ws,
+                 size_t ws_bytes, bool accept_stage) {
+  // [B, L] and [B, K, L, V] arrays are empty when L == 0, so their pointers may then be NULL.
+  if (!target || (L > 0 && !draft)) return SPEC_ERR_ARG;
+  if (accept_stage && (!g || !accept_len || !out_tokens || (L > 0 && (!tokens || !u)))) return SPEC_ERR_ARG;
+  if (!dtype_ok(dtype) || V < 1 || V > 0x7fffffffLL || !(T > 0.f) || !std::isfinite(T)) return SPEC_ERR_ARG;
+  if (B < 1 || L < 0 || K < 1) return SPEC_ERR_ARG;
+  if (!verify_shape_ok(B, L, K)) return SPEC_ERR_UNSUPPORTED;
+  if (accept_stage && K > 1 && !mix_w) return SPEC_ERR_ARG;
+  if (!ws) return SPEC_ERR_WORKSPACE;
+  if (ws_bytes < verify_layout(B, L, K, V).total) return SPEC_ERR_WORKSPACE;
+  const int es = esize(dtype);
+  if (!aligned(target, es) || !aligned(draft, es) || !aligned(g, 4) || !aligned(u, 4) || !aligned(tokens, 4) ||
+      !aligned(accept_len, 4) || !aligned(out_tokens, 4) || !aligned(ws, 16) || !aligned(row_off, 4) ||
+      !aligned(vlen, 4) || !aligned(mix_w, 4))
+    return SPEC_ERR_ARG;
+  return SPEC_OK;
+}
+
+// The statistics stage's vector decision; the accept stage must use the same
+// units per row and grid to find the partials.
+bool stats_vec(const void* target, const void* draft, int dtype, int64_t V) {
+  return (V * esize(dtype)) % 16 == 0 && aligned(target, 16) && aligned(draft, 16);
+}
+
+int launch_stats_stage(const void* target, const int32_t* row_off, const void* draft, int K, int dtype,
+                       const int32_t* vlen, int B, int L, int64_t V, float T, void* ws, cudaStream_t st) {
+  if (L == 0) return SPEC_OK;
+  const bool vec = stats_vec(target, draft, dtype, V);
+  const VerifyLayout lay = verify_layout(B, L, K, V);
+  RowSpace rs = {};
+  rs.target = target;
+  rs.draft = draft;
+  rs.row_off = row_off;
+  rs.vlen = vlen;
+  rs.stride = V;
+  rs.rows = 0;
+  rs.B = B;
+  rs.L = L;
+  rs.K = K;
+  rs.verify = 1;
+  const int G = stats_grid(dtype, vec, static_cast<int64_t>(B) * (K + 1) * L * units_per_row(V, dtype, vec));
+  return map_cuda(launch_row_stats(rs, dtype, vec, V, T, G, reinterpret_cast<float2*>(static_cast<char*>(ws) + lay.rpart), st));
+}
+
+int launch_accept_stage(const void* target, const int32_t* row_off, const void* draft, const float* mix_w, int K,
+                        int dtype, const int32_t* tokens, const int32_t* vlen, const float* u, const float* g, int B,
+                        int L, int64_t V, float T, int32_t* accept_len, int32_t* out_tokens, void* ws,
+                        cudaStream_t st) {
+  const bool vec = stats_vec(target, draft, dtype, V);
+  const bool vec_term = vec && aligned(g, 16);
+  const VerifyLayout lay = verify_layout(B, L, K, V);
+  char* w = static_cast<char*>(ws);
+  VerifyArgs a = {};
+  a.target = target;
+  a.row_off = row_off;
+  a.draft = draft;
+  a.mix_w = mix_w;
+  a.tokens = tokens;
+  a.vlen = vlen;
+  a.u = u;
+  a.g = g;
+  a.B = B;
+  a.L = L;
+  a.K = K;
+  a.V = V;
+  a.T = T;
+  a.accept_len = accept_len;
+  a.out_tokens = out_tokens;
+  a.status = reinterpret_cast<int*>(w);
+  a.tickets = reinterpret_cast<int*>(w + lay.tickets);
+  a.tpart = reinterpret_cast<TermPart*>(w + lay.tpart);
+  a.rpart = reinterpret_cast<const float2*>(w + lay.rpart);
+  a.Vu = units_per_row(V, dtype, vec);
+  a.G = stats_grid(dtype, vec, static_cast<int64_t>(B) * (K + 1) * L * a.Vu);
+  // Blocks per request for the terminal row: about two waves over the SMs,
+  // at least 256 units of the row per block.
+  const int64_t term_units = vec_term ? V / (16 / esize(dtype)) : V;
+  const int64_t p_sm = (2 * static_cast<int64_t>(sm_count()) + B - 1) / B;
+  a.P = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({p_sm, kPMax, term_units / kThreads})));
+  return map_cuda(launch_accept_sample(a, dtype, vec_term, st));
+}
+
+// The one-kernel path needs the vector path for every operand, V a multiple
+// of 8 and a terminal split that fits its stage ring.
+bool fused_ok(const void* target, const void* draft, const float* g, int dtype, int B, int L, int K, int64_t V) {
+  return L >= 1 && B <= kFusedMaxB && V % 8 == 0 && stats_vec(target, draft, dtype, V) && aligned(g, 16) &&
+         fused_pt(V, dtype, K) <= kFusedPtMax;
+}
+
+int launch_fused_stage(const void* target, const int32_t* row_off, const void* draft, const float* mix_w, int K,
+                       int dtype, const int32_t* tokens, const int32_t* vlen, const float* u, const float* g, int B,
+                       int L, int64_t V, float T, int32_t* accept_len, int32_t* out_tokens, void* ws,
+                       cudaStream_t st) {
+  const VerifyLayout lay = verify_layout(B, L, K, V);
+  char* w = static_cast<char*>(ws);
+  FusedArgs a = {};
+  a.target = target;
+  a.row_off = row_off;
+  a.draft = draft;
+  a.mix_w = mix_w;
+  a.tokens = tokens;
+  a.vlen = vlen;
+  a.u = u;
+  a.g = g;
+  a.B = B;
+  a.L = L;
+  a.K = K;
+  a.V = V;
+  a.T = T;
+  a.k = static_cast<float>(1.4426950408889634 / static_cast<double>(T));
+  a.accept_len = accept_len;
+  a.out_tokens = out_tokens;
+  a.status = reinterpret_cast<int*>(w);
+  a.ctl = reinterpret_cast<int*>(w + lay.ctl);
+  a.req_cnt = reinterpret_cast<int*>(w + lay.req_cnt);
+  a.tterm = reinterpret_cast<int*>(w + lay.tterm);
+  a.dready = reinterpret_cast<int*>(w + lay.dready);
+  a.dec = reinterpret_cast<Decision*>(w + lay.dec);
+  a.tpart = reinterpret_cast<TermPart*>(w + lay.tpart_f);
+  a.xg = reinterpret_cast<float*>(w + lay.xg);
+  a.part = reinterpret_cast<float2*>(w + lay.part_f);
+  a.cpr = fused_cpr(V, dtype);
+  a.Vu = units_per_row(V, dtype, true);
+  a.Pt = fused_pt(V, dtype, K);
+  a.Vq = V / 8;
+  return map_cuda(launch_fused(a, dtype, sm_count(), st));
+}
+
+int verify_common(const void* target, const int32_t* row_off, const void* draft, const float* mix_w, int K,
+                  int dtype, const int32_t* tokens, const int32_t* vlen, const float* u, const float* g, int B,
+                  int L, int64_t V, float T, int32_t* accept_len, int32_t* out_tokens, void* ws, size_t ws_bytes,
+                  cudaStream_t st) {
+  int e = verify_check(target, row_off, draft, mix_w, K, dtype, tokens, vlen, u, g, B, L, V, T, accept_len,
+                       out_tokens, ws, ws_bytes, true);
+  if (e) return e;
+  if (fused_ok(target, draft, g, dtype, B, L, K, V))
+    return launch_fused_stage(target, row_off, draft, mix_w, K, dtype, tokens, vlen, u, g, B, L, V, T, accept_len,
+                              out_tokens, ws, st);
+  e = launch_stats_stage(target, row_off, draft, K, dtype, vlen, B, L, V, T, ws, st);
+  if (e) return e;
+  return launch_accept_stage(target, row_off, draft, mix_w, K, dtype, tokens, vlen, u, g, B, L, V, T, accept_len,
+                             out_tokens, ws, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* spec_status_string(int status) {
+  switch (status) {
+    case SPEC_OK: return "SPEC_OK";
+    case SPEC_ERR_ARG: return "SPEC_ERR_ARG: invalid argument (null pointer, size, alignment, T or budget)";
+    case SPEC_ERR_UNSUPPORTED: return "SPEC_ERR_UNSUPPORTED: shape outside the supported limits";
+    case SPEC_ERR_CUDA: return "SPEC_ERR_CUDA: a kernel launch failed";
+    case SPEC_ERR_WORKSPACE: return "SPEC_ERR_WORKSPACE: workspace missing or too small";
+    default: return "unknown spec_status";
+  }
+}
+
+size_t spec_softmax_workspace_size(int64_t rows) {
+  if (rows < 0 || rows > (int64_t{1} << 31)) return 0;
+  return kHeader + align256((static_cast<size_t>(kGMax) + static_cast<size_t>(rows)) * sizeof(float2));
+}
+
+size_t spec_verify_workspace_size(int B, int L, int K, int64_t V) {
+  if (!verify_shape_ok(B, L, K) || V < 1 || V > 0x7fffffffLL) return 0;
+  return verify_layout(B, L, K, V).total;
+}
+
+size_t spec_dvl_workspace_size(int B) {
+  if (B < 1 || B > SPEC_MAX_B) return 0;
+  return 2 * kHeader;
+}
+
+int spec_workspace_init(void* workspace, size_t ws_bytes, spec_stream_t stream) {
+  if (!workspace || ws_bytes == 0) return SPEC_ERR_ARG;
+  return map_cuda(cudaMemsetAsync(workspace, 0, ws_bytes, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int spec_softmax_T(const void* logits, int dtype, int64_t rows, int64_t V, int64_t row_stride, float T,
+                   float* row_max, float* row_lse, float* probs, void* workspace, size_t ws_bytes,
+                   spec_stream_t stream) {
+  if (!logits || !row_max || !row_lse) return SPEC_ERR_ARG;
+  if (!dtype_ok(dtype) || rows < 0 || V < 1 || V > 0x7fffffffLL || row_stride < V || !(T > 0.f) ||
+      !std::isfinite(T))
+    return SPEC_ERR_ARG;
+  if (rows > (int64_t{1} << 31)) return SPEC_ERR_UNSUPPORTED;
+  if (!workspace) return SPEC_ERR_WORKSPACE;
+  if (ws_bytes < spec_softmax_workspace_size(rows)) return SPEC_ERR_WORKSPACE;
+  const int es = esize(dtype);
+  if (!aligned(logits, es) || !aligned(row_max, 4) || !aligned(row_lse, 4) || (probs && !aligned(probs, 4)) ||
+      !aligned(workspace, 16))
+    return SPEC_ERR_ARG;
+  if (rows == 0) return SPEC_OK;
+  const bool vec = (V * es) % 16 == 0 && (row_stride * es) % 16 == 0 && aligned(logits, 16) &&
+                   (!probs || aligned(probs, 16));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float2* part = reinterpret_cast<float2*>(static_cast<char*>(workspace) + kHeader);
+  const int64_t Vu = units_per_row(V, dtype, vec);
+  const int G = stats_grid(dtype, vec, rows * Vu);
+  RowSpace rs = {};
+  rs.target = logits;
+  rs.stride = row_stride;
+  rs.rows = rows;
+  rs.verify = 0;
+  int e = map_cuda(launch_row_stats(rs, dtype, vec, V, T, G, part, st));
+  if (e) return e;
+  return map_cuda(
+      launch_softmax_finalize(logits, dtype, vec, rows, V, row_stride, T, G, part, row_max, row_lse, probs, st));
+}
+
+int spec_verify_block(const void* target_logits, const int32_t* target_row_off, const void* draft_logits, int dtype,
+                      const int32_t* draft_tokens, const int32_t* verify_len, const float* uniforms,
+                      const float* gumbel, int B, int L, int64_t V, float T, int32_t* accept_len,
+                      int32_t* out_tokens, void* workspace, size_t ws_bytes, spec_stream_t stream) {
+  return verify_common(target_logits, target_row_off, draft_logits, nullptr, 1, dtype, draft_tokens, verify_len,
+                       uniforms, gumbel, B, L, V, T, accept_len, out_tokens, workspace, ws_bytes,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+int spec_verify_mixture(const void* target_logits, const int32_t* target_row_off, const void* draft_logits,
+                        const float* mix_weights, int K, int dtype, const int32_t* draft_tokens,
+                        const int32_t* verify_len, const float* uniforms, const float* gumbel, int B, int L,
+                        int64_t V, float T, int32_t* accept_len, int32_t* out_tokens, void* workspace,
+                        size_t ws_bytes, spec_stream_t stream) {
+  if (!mix_weights) return SPEC_ERR_ARG;
+  return verify_common(target_logits, target_row_off, draft_logits, mix_weights, K, dtype, draft_tokens, verify_len,
+                       uniforms, gumbel, B, L, V, T, accept_len, out_tokens, workspace, ws_bytes,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+int spec_verify_window_stats(const void* target_logits, const int32_t* target_row_off, const void* draft_logits,
+                             int K, int dtype, const int32_t* verify_len, int B, int L, int64_t V, float T,
+                             void* workspace, size_t ws_bytes, spec_stream_t stream) {
+  const int e = verify_check(target_logits, target_row_off, draft_logits, nullptr, K, dtype, nullptr, verify_len,
+                             nullptr, nullptr, B, L, V, T, nullptr, nullptr, workspace, ws_bytes, false);
+  if (e) return e;
+  return launch_stats_stage(target_logits, target_row_off, draft_logits, K, dtype, verify_len, B, L, V, T, workspace,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+int spec_verify_accept(const void* target_logits, const int32_t* target_row_off, const void* draft_logits,
+                       const float* mix_weights, int K, int dtype, const int32_t* draft_tokens,
+                       const int32_t* verify_len, const float* uniforms, const float* gumbel, int B, int L, int64_t V,
+                       float T, int32_t* accept_len, int32_t* out_tokens, void* workspace, size_t ws_bytes,
+                       spec_stream_t stream) {
+  const int e = verify_check(target_logits, target_row_off, draft_logits, mix_weights, K, dtype, draft_tokens,
+                             verify_len, uniforms, gumbel, B, L, V, T, accept_len, out_tokens, workspace, ws_bytes,
+                             true);
+  if (e) return e;
+  return launch_accept_stage(target_logits, target_row_off, draft_logits, mix_weights, K, dtype, draft_tokens,
+                             verify_len, uniforms, gumbel, B, L, V, T, accept_len, out_tokens, workspace,
+                             reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dvl_allocate_pack(const float* scores, int B, int L, int budget, int32_t* verify_len, int32_t* offsets,
+                      int32_t* slot_map, const void* dense_target, void* packed_target, int dtype, int64_t V,
+                      void* workspace, size_t ws_bytes, spec_stream_t stream) {
+  if (!scores || !verify_len || !offsets) return SPEC_ERR_ARG;
+  if (B < 1 || L < 0 || budget < B) return SPEC_ERR_ARG;
+  if (B > SPEC_MAX_B || L > SPEC_MAX_L || static_cast<int64_t>(B) * L > SPEC_MAX_DVL_ELEMS)
+    return SPEC_ERR_UNSUPPORTED;
+  const bool pack = dense_target || packed_target;
+  if (pack && (!dense_target || !packed_target || !dtype_ok(dtype) || V < 1 || V > 0x7fffffffLL))
+    return SPEC_ERR_ARG;
+  if (!aligned(scores, 4) || !aligned(verify_len, 4) || !aligned(offsets, 4) || (slot_map && !aligned(slot_map, 4)))
+    return SPEC_ERR_ARG;
+  if (pack && (!aligned(dense_target, esize(dtype)) || !aligned(packed_target, esize(dtype)))) return SPEC_ERR_ARG;
+  if (!workspace) return SPEC_ERR_WORKSPACE;
+  if (ws_bytes < spec_dvl_workspace_size(B) || !aligned(workspace, 16)) return SPEC_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(workspace);
+  int* ticket = reinterpret_cast<int*>(static_cast<char*>(workspace) + kHeader);
+  int e = map_cuda(launch_dvl(scores, B, L, budget, verify_len, offsets, slot_map, status, ticket, st));
+  if (e || !pack) return e;
+  return map_cuda(launch_pack(dense_target, packed_target, dtype, B, L, V, budget, offsets, st));
+}
+
+}  // extern "C"

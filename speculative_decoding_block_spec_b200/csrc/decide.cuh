@@ -1,0 +1,153 @@
+// The per-request accept decision, shared by both verify paths.
+//
+// Speculative sampling with rejection correction ("DBLAST: Dependent Block
+// Drafting for Stochastic Speculative Decoding", Pith review, "Assumptions"):
+// position i is accepted iff u_i < min(1, p_i(x_i) / q_i(x_i)); the verifier
+// stops at the first rejection. For a latent-mixture draft ("What carries the
+// argument", Eq. 5) q_i is the mixture marginal under the category posterior
+// pi_i(z) ∝ q(z|y) prod_{k<i} q_k(x_k|y,z).
+#pragma once
+
+#include "common.cuh"
+
+namespace specv {
+
+constexpr int kMaxL = 32;
+constexpr int kMaxK = 8;
+constexpr int kMaxRows = (kMaxK + 1) * kMaxL;
+
+// Inputs of one request's decision, in shared memory. Row q of the request:
+// q < ell is target position q; q = ell + z*ell + i is draft (z, i).
+struct DecideIn {
+  const float* xg;   // raw logit at the drafted token, per row
+  const float* m;    // row max of raw logits
+  const float* s;    // sum 2^((x - m) log2e / T)
+  const int* x;      // drafted tokens [ell]
+  int ell, K, L;
+  float T;
+};
+
+// Terminal-row parameters: p(v) = 2^((x_t - mt) k) * ct, q(v) = sum_z 2^((x_z - mz) k) * cz.
+struct DecideOut {
+  int j;
+  int bad;            // a non-finite posterior or ratio at or before j
+  float ct, mt;
+  float cz[kMaxK], mz[kMaxK];
+};
+
+// Run by the 32 lanes of one warp (lane i tests position i) in fp64: the
+// normalisers are the only fp32 quantities. u, mix_w: this request's rows.
+__device__ __forceinline__ DecideOut decide_warp(const DecideIn& in, const float* u, const float* mix_w) {
+  const int lane = threadIdx.x & 31;
+  const int ell = in.ell, K = in.K;
+  const double T = static_cast<double>(in.T);
+  const bool act = lane < ell;
+  double lp = 0.0, lqz[kMaxK];
+#pragma unroll
+  for (int z = 0; z < kMaxK; ++z) lqz[z] = 0.0;
+  if (act) {
+    lp = (static_cast<double>(in.xg[lane]) - static_cast<double>(in.m[lane])) / T -
+         log(static_cast<double>(in.s[lane]));
+#pragma unroll
+    for (int z = 0; z < kMaxK; ++z) {
+      if (z < K) {
+        const int q = ell + z * ell + lane;
+        lqz[z] = (static_cast<double>(in.xg[q]) - static_cast<double>(in.m[q])) / T -
+                 log(static_cast<double>(in.s[q]));
+      }
+    }
+  }
+  // log pi_i(z) = log w_z + sum_{k<i} log q_k(x_k|y,z) - logsumexp_z(.); for K = 1
+  // this is exactly 0 and q_i = q_i(.|y), the independent proposal.
+  double lpi[kMaxK];
+  double amax = -INFINITY;
+#pragma unroll
+  for (int z = 0; z < kMaxK; ++z) {
+    lpi[z] = 0.0;
+    if (z < K) {
+      double v = __shfl_up_sync(0xffffffffu, lqz[z], 1);
+      if (lane == 0) v = 0.0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const double t = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += t;
+      }
+      const double lw = mix_w ? log(static_cast<double>(mix_w[z])) : 0.0;
+      lpi[z] = lw + v;
+      amax = fmax(amax, lpi[z]);
+    }
+  }
+  double sa = 0.0;
+#pragma unroll
+  for (int z = 0; z < kMaxK; ++z)
+    if (z < K) sa += exp(lpi[z] - amax);
+  const double norm = amax + log(sa);
+  double tmax = -INFINITY;
+#pragma unroll
+  for (int z = 0; z < kMaxK; ++z) {
+    if (z < K) {
+      lpi[z] -= norm;
+      tmax = fmax(tmax, lpi[z] + lqz[z]);
+    }
+  }
+  double st = 0.0;
+#pragma unroll
+  for (int z = 0; z < kMaxK; ++z)
+    if (z < K) st += exp(lpi[z] + lqz[z] - tmax);
+  const double lq = tmax + log(st);
+  const double rho = exp(lp - lq);
+  const bool bad = !isfinite(norm) || isnan(rho);
+  const double thr = fmin(1.0, rho);
+  const float uu = act ? u[lane] : 0.f;
+  const bool acc = static_cast<double>(uu) < thr;
+  const unsigned stop = __ballot_sync(0xffffffffu, act && (bad || !acc));
+  DecideOut o;
+  o.j = stop ? __ffs(stop) - 1 : ell;
+  o.bad = (__shfl_sync(0xffffffffu, bad ? 1 : 0, o.j & 31) && stop) ? 1 : 0;
+  o.ct = o.mt = 0.f;
+  // terminal multipliers, from lane j (residual draw)
+  const int src = o.j & 31;
+  double lpj[kMaxK];
+#pragma unroll
+  for (int z = 0; z < kMaxK; ++z) lpj[z] = __shfl_sync(0xffffffffu, z < K ? lpi[z] : 0.0, src);
+  if (o.j < ell) {
+    o.ct = static_cast<float>(1.0 / static_cast<double>(in.s[o.j]));
+    o.mt = in.m[o.j];
+#pragma unroll
+    for (int z = 0; z < kMaxK; ++z) {
+      if (z < K) {
+        const int q = ell + z * ell + o.j;
+        o.cz[z] = static_cast<float>(exp(lpj[z]) / static_cast<double>(in.s[q]));
+        o.mz[z] = in.m[q];
+      } else {
+        o.cz[z] = 0.f;
+        o.mz[z] = 0.f;
+      }
+    }
+  }
+  return o;
+}
+
+// ------------------------------------------------------------ terminal draw
+
+struct Best {
+  double score;
+  int idx;
+};
+
+// Higher score wins; equal scores go to the lower token.
+__device__ __forceinline__ void best_merge(Best& a, const Best& b) {
+  if (b.score > a.score || (b.score == a.score && b.idx >= 0 && (a.idx < 0 || b.idx < a.idx))) a = b;
+}
+
+__device__ __forceinline__ void warp_best(Best& v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    Best w;
+    w.score = __shfl_xor_sync(0xffffffffu, v.score, o);
+    w.idx = __shfl_xor_sync(0xffffffffu, v.idx, o);
+    best_merge(v, w);
+  }
+}
+
+}  // namespace specv

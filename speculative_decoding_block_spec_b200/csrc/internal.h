@@ -1,0 +1,149 @@
+// Host-side interfaces between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace specv {
+
+// The rows walked by the row-statistics kernel.
+//  plain  (verify == 0): row r at target + r * stride elements, r < rows.
+//  verify (verify == 1): request b contributes (K+1) * l_b rows, l_b =
+//    verify_len[b] (L if NULL): first target rows 0..l_b-1 (row of (b, i) is
+//    row_off[b] + i, or b*(L+1) + i when row_off is NULL), then draft rows
+//    (z, i) for z < K, i < l_b at draft + ((b*K + z)*L + i) * V.
+struct RowSpace {
+  const void* target;
+  const void* draft;
+  const int32_t* row_off;
+  const int32_t* vlen;
+  int64_t stride;
+  int64_t rows;
+  int B, L, K;
+  int verify;
+};
+
+// Per-request terminal-draw partial of one sampling block.
+struct TermPart {
+  double res_score;  // best residual score (ln r + g), -inf if none
+  double bon_score;  // best bonus-rule score (x / T + g)
+  int res_idx;       // its token, -1 if none
+  int bon_idx;
+  int pad[2];
+};
+
+// Everything the accept/sample kernel reads.
+struct VerifyArgs {
+  const void* target;
+  const int32_t* row_off;
+  const void* draft;
+  const float* mix_w;       // nullable: w = 1 (K == 1)
+  const int32_t* tokens;
+  const int32_t* vlen;      // nullable
+  const float* u;
+  const float* g;
+  int B, L, K;
+  int64_t V;
+  float T;
+  int32_t* accept_len;
+  int32_t* out_tokens;
+  int* status;
+  int* tickets;             // [B], self-resetting
+  TermPart* tpart;          // [B * P]
+  const float2* rpart;      // row-statistics partials
+  int G;                    // row-statistics grid size
+  int64_t Vu;               // row-statistics units per row
+  int P;                    // sampling blocks per request
+};
+
+// Per-request decision published by the fused kernel's decider block.
+struct Decision {
+  int j, flags, ell, pad;
+  float ct, mt, pad2[2];
+  float cz[8], mz[8];
+};
+
+// Everything the fused verify kernel reads and writes.
+struct FusedArgs {
+  const void* target;
+  const int32_t* row_off;
+  const void* draft;
+  const float* mix_w;
+  const int32_t* tokens;
+  const int32_t* vlen;
+  const float* u;
+  const float* g;
+  int B, L, K;
+  int64_t V;
+  float T;
+  float k;                  // log2(e) / T
+  int32_t* accept_len;
+  int32_t* out_tokens;
+  int* status;
+  int* ctl;                 // [0] epoch, [1] work counter, [2] exit counter
+  int* req_cnt;             // [B] statistics chunks done, reset by the decider
+  int* tterm;               // [B] terminal chunks done, reset by the last one
+  int* dready;              // [B] epoch + 1 once the decision is published
+  Decision* dec;            // [B]
+  TermPart* tpart;          // [B * Pt]
+  float* xg;                // [rows] logit at the drafted token
+  float2* part;             // [rows * cpr] statistics partials
+  int cpr;                  // statistics chunks per row
+  int64_t Vu;               // 16-byte units per row
+  int Pt;                   // terminal chunks per request
+  int64_t Vq;               // 8-element groups per row
+};
+
+// Fused-path geometry (host and device agree on these).
+constexpr int kFusedStageBytes = 32768;
+constexpr int kFusedStages = 6;
+constexpr int kFusedMaxB = 512;
+constexpr int kFusedPtMax = 192;
+int fused_cpr(int64_t V, int dtype);
+int fused_pt(int64_t V, int dtype, int K);
+size_t fused_smem_bytes(int B);
+cudaError_t launch_fused(const FusedArgs& a, int dtype, int grid, cudaStream_t st);
+
+// Units of work per row: 16-byte vectors on the vector path, else elements.
+inline int64_t units_per_row(int64_t V, int dtype, bool vec) {
+  return vec ? V * (dtype == 0 ? 4 : 2) / 16 : V;
+}
+
+// Grid size of the persistent row-statistics kernel for up to max_units units.
+int stats_grid(int dtype, bool vec, int64_t max_units);
+
+cudaError_t launch_row_stats(const RowSpace& rs, int dtype, bool vec, int64_t V, float T, int G,
+                             float2* part, cudaStream_t st);
+
+cudaError_t launch_softmax_finalize(const void* logits, int dtype, bool vec, int64_t rows, int64_t V,
+                                    int64_t stride, float T, int G, const float2* part, float* row_max,
+                                    float* row_lse, float* probs, cudaStream_t st);
+
+cudaError_t launch_accept_sample(const VerifyArgs& a, int dtype, bool vec, cudaStream_t st);
+
+cudaError_t launch_dvl(const float* scores, int B, int L, int budget, int32_t* verify_len,
+                       int32_t* offsets, int32_t* slot_map, int* status, int* ticket,
+                       cudaStream_t st);
+
+cudaError_t launch_pack(const void* dense, void* packed, int dtype, int B, int L, int64_t V,
+                        int budget, const int32_t* offsets, cudaStream_t st);
+
+// Launch helper: programmatic stream serialization lets the grid start while
+// its predecessor drains; each kernel calls griddepcontrol.wait first.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+}  // namespace specv

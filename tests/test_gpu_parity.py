@@ -1,0 +1,303 @@
+"""GPU <-> oracle parity through the C ABI (needs a B200).
+
+Every input is seeded and synthetic (speculative_decoding_block_spec_b200.synth).
+Decisions (accepted lengths, tokens, verify lengths, offsets, slot maps,
+packed rows) must match bit for bit, under the low-margin rule of
+tests/parity_util.py; softmax maxima, normalisers and probabilities within
+1e-5 relative.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import speculative_decoding_block_spec_b200 as specv
+from speculative_decoding_block_spec_b200 import synth
+from speculative_decoding_block_spec_b200.synth import f32_to_bf16_bits
+
+from parity_util import check_verify, logits_to_torch, to_torch
+
+pytestmark = pytest.mark.gpu
+NT = oracle.n_cores()
+
+
+@pytest.fixture(scope="module", autouse=True)
+def side_stream():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    specv.lib()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        yield s
+    s.synchronize()
+
+
+def _cpu(t):
+    torch.cuda.current_stream().synchronize()
+    return t.cpu().numpy()
+
+
+# ----------------------------------------------------------------- softmax_T
+
+@pytest.mark.parametrize("rows,V,dtype,T,probs", [
+    (6, 64, "f32", 1.0, True),
+    (9, 1001, "f32", 1.5, True),        # scalar path (V*4 not a multiple of 16)
+    (5, 1001, "bf16", 0.7, True),       # scalar path
+    (1, 8, "bf16", 1.0, True),
+    (300, 4096, "bf16", 1.0, True),     # many rows per block
+    (40, 151936, "bf16", 1.0, False),
+    (12, 151936, "bf16", 1.5, True),
+    (3, 151936, "f32", 1.0, True),
+])
+def test_softmax_parity(rows, V, dtype, T, probs):
+    rng = np.random.default_rng(rows * 7 + V)
+    x = rng.standard_normal((rows, V)).astype(np.float32) * 2
+    x[:, -1] += 9.0                      # the peak sits in the final chunk
+    x[0, 0] += 12.0
+    xs = f32_to_bf16_bits(x) if dtype == "bf16" else x
+    ref = oracle.softmax_T(xs, T, probs=probs)
+    got = specv.softmax_T(logits_to_torch(xs), T, probs=probs)
+    np.testing.assert_allclose(_cpu(got[0]), ref[0], rtol=1e-5, atol=0)
+    np.testing.assert_allclose(_cpu(got[1]), ref[1], rtol=1e-5, atol=1e-6)
+    if probs:
+        np.testing.assert_allclose(_cpu(got[2]), ref[2], rtol=1e-5, atol=1e-37)
+
+
+# ------------------------------------------------------------ the workloads
+
+def _verify(d, x, T, verify_len=None, target=None, row_off=None, path="fused"):
+    """One verification through the C ABI. path 'fused' is the public one-call
+    entry point (one persistent kernel when the shapes allow it); 'split' runs
+    its two stages, spec_verify_window_stats then spec_verify_accept."""
+    tgt = d["target"] if target is None else target
+    mix = d.get("mix_w") if x.w.K > 1 else None
+    if path == "split":
+        B, L = d["tokens"].shape
+        ws = specv.Workspace(specv.verify_workspace_size(B, L, x.w.K, x.w.V))
+        specv.spec_verify_window_stats(tgt, d["draft"], T, ws, K=x.w.K, L=L, verify_len=verify_len,
+                                       target_row_off=row_off)
+        return specv.spec_verify_accept(tgt, d["draft"], d["tokens"], d["u"], d["g"], T, ws, mix_w=mix,
+                                        verify_len=verify_len, target_row_off=row_off)
+    if x.w.K == 1:
+        return specv.spec_verify_block(tgt, d["draft"], d["tokens"], d["u"], d["g"], T, verify_len=verify_len,
+                                       target_row_off=row_off)
+    return specv.spec_verify_mixture(tgt, d["draft"], d["mix_w"], d["tokens"], d["u"], d["g"], T,
+                                     verify_len=verify_len, target_row_off=row_off)
+
+
+PATHS = ["fused", "split"]
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("cid", [1, 2, 3])
+def test_dense_workloads(cid, path):
+    x = synth.workload_inputs(cid)
+    ref = oracle.verify(x.target, x.draft, x.tokens, x.u, x.g, x.w.T, mix_w=x.mix_w, n_threads=NT, diag=True)
+    d = to_torch(x)
+    acc, out = _verify(d, x, x.w.T, path=path)
+    check_verify(_cpu(acc), _cpu(out), ref)
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("cid", [4, 5])
+def test_dvl_packed_workloads(cid, path):
+    x = synth.workload_inputs(cid)
+    w = x.w
+    rd = oracle.dvl_allocate(x.scores, w.budget)
+    packed_ref = oracle.pack(x.target, rd["verify_len"], rd["offsets"], w.budget)
+    ref = oracle.verify(packed_ref, x.draft, x.tokens, x.u, x.g, w.T, mix_w=x.mix_w, n_threads=NT, diag=True,
+                        verify_len=rd["verify_len"], target_row_off=rd["offsets"][:w.B])
+    d = to_torch(x)
+    packed = torch.zeros((w.budget, w.V), dtype=d["target"].dtype, device="cuda")
+    vl, off, sm = specv.dvl_allocate_pack(d["scores"], w.budget, dense_target=d["target"], packed_target=packed)
+    np.testing.assert_array_equal(_cpu(vl), rd["verify_len"])
+    np.testing.assert_array_equal(_cpu(off), rd["offsets"])
+    np.testing.assert_array_equal(_cpu(sm), rd["slot_map"])
+    pk = _cpu(packed.view(torch.int16)).view(np.uint16)
+    np.testing.assert_array_equal(pk[:rd["offsets"][-1]], packed_ref[:rd["offsets"][-1]])
+    acc, out = _verify(d, x, w.T, verify_len=vl, target=packed, row_off=off[:w.B], path=path)
+    check_verify(_cpu(acc), _cpu(out), ref, verify_len=rd["verify_len"])
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("seed", range(6))
+def test_seed_sweep_block_and_mixture(seed, path):
+    K = 1 if seed % 2 == 0 else 3
+    x = synth.custom(B=8, L=16, V=32768, K=K, T=1.0 + 0.25 * (seed % 3), dtype="bf16", n_peaks=8, peak=6.0,
+                     draft_sigma=0.7, seed=seed, cid=200 + seed)
+    vl = np.random.default_rng(seed).integers(0, 17, size=8).astype(np.int32)
+    ref = oracle.verify(x.target, x.draft, x.tokens, x.u, x.g, x.w.T, mix_w=x.mix_w, verify_len=vl,
+                        n_threads=NT, diag=True)
+    d = to_torch(x)
+    acc, out = _verify(d, x, x.w.T, verify_len=torch.from_numpy(vl).cuda(), path=path)
+    check_verify(_cpu(acc), _cpu(out), ref, verify_len=vl)
+
+
+# -------------------------------------------------------------- identities
+
+def test_k1_mixture_is_bit_identical_to_block():
+    x = synth.custom(B=6, L=16, V=151936, K=1, dtype="bf16", n_peaks=32, peak=8.0, seed=11, cid=300)
+    d = to_torch(x)
+    a1, o1 = specv.spec_verify_block(d["target"], d["draft"], d["tokens"], d["u"], d["g"], 1.0)
+    a2, o2 = specv.spec_verify_mixture(d["target"], d["draft"][:, None].contiguous(),
+                                       torch.ones((6, 1), dtype=torch.float32, device="cuda"),
+                                       d["tokens"], d["u"], d["g"], 1.0)
+    assert torch.equal(a1, a2) and torch.equal(o1, o2)
+
+
+def test_q_equals_p_accepts_everything():
+    x = synth.custom(B=4, L=16, V=151936, K=1, dtype="bf16", n_peaks=32, peak=8.0, seed=12, cid=301)
+    x.draft = x.target[:, :16].copy()
+    vl = np.array([16, 5, 0, 1], np.int32)
+    ref = oracle.verify(x.target, x.draft, x.tokens, x.u, x.g, 1.0, verify_len=vl, n_threads=NT, diag=True)
+    d = to_torch(x)
+    acc, out = specv.spec_verify_block(d["target"], d["draft"], d["tokens"], d["u"], d["g"], 1.0,
+                                       verify_len=torch.from_numpy(vl).cuda())
+    np.testing.assert_array_equal(_cpu(acc), vl)
+    check_verify(_cpu(acc), _cpu(out), ref, verify_len=vl)
+
+
+def test_one_hot_target_and_vocab_edge_tokens():
+    rng = np.random.default_rng(13)
+    B, L, V = 4, 6, 151936
+    t = rng.standard_normal((B, L + 1, V)).astype(np.float32)
+    star = np.array([[0, V - 1, 5, V - 2, 77, 1000, V - 1]] * B)
+    for b in range(B):
+        for i in range(L + 1):
+            t[b, i, star[b, i]] = 1000.0
+    dr = rng.standard_normal((B, L, V)).astype(np.float32)
+    tokens = np.zeros((B, L), np.int32)
+    tokens[1] = V - 1
+    tokens[2, ::2] = V - 1
+    u = rng.random((B, L), dtype=np.float32)
+    g = synth.gumbel(rng, (B, L + 1, V)).astype(np.float32)
+    for dtype in ("f32", "bf16"):
+        tt = f32_to_bf16_bits(t) if dtype == "bf16" else t
+        dd = f32_to_bf16_bits(dr) if dtype == "bf16" else dr
+        ref = oracle.verify(tt, dd, tokens, u, g, 1.0, n_threads=NT, diag=True)
+        acc, out = specv.spec_verify_block(logits_to_torch(tt), logits_to_torch(dd), torch.from_numpy(tokens).cuda(),
+                                           torch.from_numpy(u).cuda(), torch.from_numpy(g).cuda(), 1.0)
+        check_verify(_cpu(acc), _cpu(out), ref)
+        # rows where the drafted token is not the one-hot token reject at 0 and emit the one-hot token
+        o = _cpu(out)
+        for b in range(B):
+            if tokens[b, 0] != star[b, 0]:
+                assert o[b, 0] == star[b, 0]
+
+
+def test_exact_ties_go_to_lowest_index():
+    B, L, V = 2, 2, 4096
+    target = np.zeros((B, L + 1, V), np.float32)          # uniform target rows
+    draft = np.zeros((B, L, V), np.float32)
+    draft[0, 0, 100] = 6.0                                  # request 0 drafts an over-weighted token
+    tokens = np.array([[100, 0], [3, 4]], np.int32)
+    u = np.array([[0.999, 0.5], [0.5, 0.5]], np.float32)
+    g = np.zeros((B, L + 1, V), np.float32)
+    acc, out = specv.spec_verify_block(*(torch.from_numpy(a).cuda() for a in (target, draft, tokens, u, g)), 1.0)
+    acc, out = _cpu(acc), _cpu(out)
+    # request 0: rejected at 0; residual mass is equal on every token but 100 -> lowest index 0
+    assert acc[0] == 0 and out[0, 0] == 0
+    # request 1: q == p (uniform) -> all accepted; uniform bonus row, zero noise -> token 0
+    assert acc[1] == 2 and list(out[1]) == [3, 4, 0]
+
+
+# ----------------------------------------------------------- device errors
+
+@pytest.mark.parametrize("path", PATHS)
+def test_device_flags_and_isolation(path):
+    x = synth.custom(B=4, L=8, V=4096, K=2, dtype="bf16", n_peaks=4, peak=5.0, seed=14, cid=302)
+    x.tokens[1, 3] = 4096                        # out of range
+    x.target[3, 2, 17] = 0x7FC0                  # NaN in a tested row of request 3
+    vl = np.array([8, 8, 8, 8], np.int32)
+    ref = oracle.verify(x.target, x.draft, x.tokens, x.u, x.g, 1.0, mix_w=x.mix_w, verify_len=vl, diag=True)
+    assert ref["flags"] & oracle.FLAG_TOKEN_RANGE and ref["flags"] & oracle.FLAG_NONFINITE
+    d = to_torch(x)
+    ws = specv.Workspace(specv.verify_workspace_size(4, 8, 2, 4096))
+    if path == "split":
+        vlt = torch.from_numpy(vl).cuda()
+        specv.spec_verify_window_stats(d["target"], d["draft"], 1.0, ws, K=2, verify_len=vlt)
+        acc, out = specv.spec_verify_accept(d["target"], d["draft"], d["tokens"], d["u"], d["g"], 1.0, ws,
+                                            mix_w=d["mix_w"], verify_len=vlt)
+    else:
+        acc, out = specv.spec_verify_mixture(d["target"], d["draft"], d["mix_w"], d["tokens"], d["u"], d["g"],
+                                             1.0, verify_len=torch.from_numpy(vl).cuda(), workspace=ws)
+    st = ws.status()
+    assert st & specv.DEV_TOKEN_RANGE and st & specv.DEV_NONFINITE
+    check_verify(_cpu(acc), _cpu(out), ref, verify_len=vl)
+    # an out-of-range verify length
+    ws.init()
+    bad = torch.tensor([8, 9, -1, 0], dtype=torch.int32, device="cuda")
+    acc, out = specv.spec_verify_mixture(d["target"], d["draft"], d["mix_w"], d["tokens"], d["u"], d["g"], 1.0,
+                                         verify_len=bad, workspace=ws)
+    a = _cpu(acc)
+    assert ws.status() & specv.DEV_VERIFY_LEN
+    assert a[1] == -1 and a[2] == -1 and a[3] == 0
+
+
+def test_workspace_reuse_is_self_resetting():
+    """Many calls on one workspace, alternating the fused and the two-stage
+    paths and changing shapes within its capacity: no re-initialisation."""
+    x = synth.custom(B=5, L=16, V=65536, K=1, dtype="bf16", n_peaks=8, peak=6.0, seed=15, cid=303)
+    d = to_torch(x)
+    ws = specv.Workspace(specv.verify_workspace_size(5, 16, 2, 65536))
+    first = specv.spec_verify_block(d["target"], d["draft"], d["tokens"], d["u"], d["g"], 1.0, workspace=ws)
+    first = [t.clone() for t in first]
+    for it in range(6):
+        if it % 3 == 2:
+            specv.spec_verify_window_stats(d["target"], d["draft"], 1.0, ws)
+            again = specv.spec_verify_accept(d["target"], d["draft"], d["tokens"], d["u"], d["g"], 1.0, ws)
+        else:
+            again = specv.spec_verify_block(d["target"], d["draft"], d["tokens"], d["u"], d["g"], 1.0,
+                                            workspace=ws)
+        assert torch.equal(first[0], again[0]) and torch.equal(first[1], again[1]), it
+    vl = torch.tensor([3, 0, 16, 7, 1], dtype=torch.int32, device="cuda")
+    ref = oracle.verify(x.target, x.draft, x.tokens, x.u, x.g, 1.0, verify_len=vl.cpu().numpy(), diag=True)
+    for _ in range(3):
+        acc, out = specv.spec_verify_block(d["target"], d["draft"], d["tokens"], d["u"], d["g"], 1.0,
+                                           verify_len=vl, workspace=ws)
+        check_verify(_cpu(acc), _cpu(out), ref, verify_len=vl.cpu().numpy())
+    assert ws.status() == 0
+
+
+def test_scalar_path_odd_vocab():
+    for dtype, K in (("bf16", 1), ("f32", 2)):
+        x = synth.custom(B=3, L=5, V=1001, K=K, dtype=dtype, n_peaks=3, peak=4.0, seed=16, cid=304)
+        ref = oracle.verify(x.target, x.draft, x.tokens, x.u, x.g, 1.3, mix_w=x.mix_w, diag=True)
+        d = to_torch(x)
+        if K == 1:
+            acc, out = specv.spec_verify_block(d["target"], d["draft"], d["tokens"], d["u"], d["g"], 1.3)
+        else:
+            acc, out = specv.spec_verify_mixture(d["target"], d["draft"], d["mix_w"], d["tokens"], d["u"], d["g"], 1.3)
+        check_verify(_cpu(acc), _cpu(out), ref)
+
+
+def test_zero_length_block():
+    x = synth.custom(B=3, L=0, V=2048, K=1, dtype="bf16", seed=17, cid=305)
+    ref = oracle.verify(x.target, x.draft, x.tokens, x.u, x.g, 1.0, diag=True)
+    d = to_torch(x)
+    acc, out = specv.spec_verify_block(d["target"], d["draft"], d["tokens"], d["u"], d["g"], 1.0)
+    check_verify(_cpu(acc), _cpu(out), ref)
+
+
+# ---------------------------------------------------------------------- DVL
+
+@pytest.mark.parametrize("B,L,budget", [(1, 4, 1), (3, 4, 7), (32, 16, 272), (64, 16, 544), (16, 32, 300),
+                                        (7, 5, 100), (200, 16, 1700), (512, 32, 8000)])
+def test_dvl_parity(B, L, budget):
+    rng = np.random.default_rng(B * 1000 + L)
+    s = rng.beta(6.0, 2.0, size=(B, L)).astype(np.float32)
+    if B % 2:
+        s[:, ::3] = 0.5                            # many equal products: tie-break by (b, i)
+    ref = oracle.dvl_allocate(s, budget)
+    vl, off, sm = specv.dvl_allocate_pack(torch.from_numpy(s).cuda(), budget)
+    np.testing.assert_array_equal(_cpu(vl), ref["verify_len"])
+    np.testing.assert_array_equal(_cpu(off), ref["offsets"])
+    np.testing.assert_array_equal(_cpu(sm), ref["slot_map"])
+
+
+def test_dvl_flags_bad_scores():
+    s = torch.full((4, 4), 0.5, device="cuda")
+    s[2, 1] = 1.5
+    ws = specv.Workspace(specv.dvl_workspace_size(4))
+    specv.dvl_allocate_pack(s, 8, workspace=ws)
+    assert ws.status() & specv.DEV_SCORES
