@@ -37,7 +37,7 @@ int sm_count() {
 // Verify workspace: persistent state first (never overlapped), then scratch
 // that the fused and the two-stage paths share.
 struct VerifyLayout {
-  size_t ctl, req_cnt, tterm, dready, tickets;       // persistent counters and flags
+  size_t ctl, req_units, keys, dready, tickets;      // persistent counters and flags
   size_t tpart, rpart;                               // two-stage scratch
   size_t dec, tpart_f, xg, part_f;                   // fused scratch
   size_t total;
@@ -47,21 +47,20 @@ VerifyLayout verify_layout(int B, int L, int K, int64_t V) {
   VerifyLayout l;
   const size_t b4 = align256(static_cast<size_t>(B) * sizeof(int));
   l.ctl = kHeader;
-  l.req_cnt = l.ctl + 256;
-  l.tterm = l.req_cnt + b4;
-  l.dready = l.tterm + b4;
+  l.req_units = l.ctl + 256;
+  l.keys = l.req_units + align256(static_cast<size_t>(B) * sizeof(unsigned long long));
+  l.dready = l.keys + align256(static_cast<size_t>(2 * B) * sizeof(unsigned long long));
   l.tickets = l.dready + b4;
   const size_t scratch = l.tickets + b4;
   const size_t rows = static_cast<size_t>(B) * (K + 1) * L;
   l.tpart = scratch;
   l.rpart = l.tpart + align256(static_cast<size_t>(B) * kPMax * sizeof(TermPart));
   const size_t split_end = l.rpart + align256((static_cast<size_t>(kGMax) + rows) * sizeof(float2));
-  const size_t cpr = static_cast<size_t>(fused_cpr(std::max<int64_t>(V, 1), SPEC_F32));
   l.dec = scratch;
   l.tpart_f = l.dec + align256(static_cast<size_t>(B) * sizeof(Decision));
   l.xg = l.tpart_f + align256(static_cast<size_t>(B) * kFusedPtMax * sizeof(TermPart));
   l.part_f = l.xg + align256(rows * sizeof(float));
-  const size_t fused_end = l.part_f + align256(rows * cpr * sizeof(float2));
+  const size_t fused_end = l.part_f + align256((static_cast<size_t>(kGMax) + rows) * 16 * sizeof(float2));
   l.total = std::max(split_end, fused_end);
   return l;
 }
@@ -159,7 +158,8 @@ int launch_accept_stage(const void* target, const int32_t* row_off, const void* 
 // The one-kernel path needs the vector path for every operand, V a multiple
 // of 8 and a terminal split that fits its stage ring.
 bool fused_ok(const void* target, const void* draft, const float* g, int dtype, int B, int L, int K, int64_t V) {
-  return L >= 1 && B <= kFusedMaxB && V % 8 == 0 && stats_vec(target, draft, dtype, V) && aligned(g, 16) &&
+  return L >= 1 && B <= kFusedMaxB && V % 8 == 0 && V <= (1 << 20) && stats_vec(target, draft, dtype, V) &&
+         aligned(g, 16) &&
          fused_pt(V, dtype, K) <= kFusedPtMax;
 }
 
@@ -188,14 +188,12 @@ int launch_fused_stage(const void* target, const int32_t* row_off, const void* d
   a.out_tokens = out_tokens;
   a.status = reinterpret_cast<int*>(w);
   a.ctl = reinterpret_cast<int*>(w + lay.ctl);
-  a.req_cnt = reinterpret_cast<int*>(w + lay.req_cnt);
-  a.tterm = reinterpret_cast<int*>(w + lay.tterm);
+  a.req_units = reinterpret_cast<unsigned long long*>(w + lay.req_units);
+  a.keys = reinterpret_cast<unsigned long long*>(w + lay.keys);
   a.dready = reinterpret_cast<int*>(w + lay.dready);
   a.dec = reinterpret_cast<Decision*>(w + lay.dec);
-  a.tpart = reinterpret_cast<TermPart*>(w + lay.tpart_f);
   a.xg = reinterpret_cast<float*>(w + lay.xg);
   a.part = reinterpret_cast<float2*>(w + lay.part_f);
-  a.cpr = fused_cpr(V, dtype);
   a.Vu = units_per_row(V, dtype, true);
   a.Pt = fused_pt(V, dtype, K);
   a.Vq = V / 8;

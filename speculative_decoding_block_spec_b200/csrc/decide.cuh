@@ -35,9 +35,107 @@ struct DecideOut {
   float cz[kMaxK], mz[kMaxK];
 };
 
-// Run by the 32 lanes of one warp (lane i tests position i) in fp64: the
-// normalisers are the only fp32 quantities. u, mix_w: this request's rows.
+// Run by the 32 lanes of one warp (lane i tests position i). A fast fp32
+// pass computes every ratio rho_i; only when some tested lane lies close to
+// its threshold (|u_i - min(1, rho_i)| below 1e-5 for independent drafts,
+// 2e-4 with a posterior, i.e. 10x the fp32 error) or meets a non-finite value
+// does the warp redo the decisions in fp64, where the normalisers are the
+// only fp32 quantities. u, mix_w: this request's rows.
+__device__ __forceinline__ DecideOut decide_warp_fp64(const DecideIn& in, const float* u, const float* mix_w);
+
 __device__ __forceinline__ DecideOut decide_warp(const DecideIn& in, const float* u, const float* mix_w) {
+  const int lane = threadIdx.x & 31;
+  const int ell = in.ell, K = in.K;
+  const bool act = lane < ell;
+  const float invT = 1.f / in.T;
+  const float uu = act ? u[lane] : 0.f;
+  float rho = 1.f, lpi[kMaxK];
+  bool finite = true;
+#pragma unroll
+  for (int z = 0; z < kMaxK; ++z) lpi[z] = 0.f;
+  if (K == 1) {
+    // rho = exp(((x_t - m_t) - (x_d - m_d)) / T + log(s_d / s_t))
+    if (act) {
+      const int q = ell + lane;
+      const float d = ((in.xg[lane] - in.m[lane]) - (in.xg[q] - in.m[q])) * invT + logf(in.s[q] / in.s[lane]);
+      rho = expf(d);
+      finite = isfinite(d) && isfinite(in.xg[q]) && isfinite(in.xg[lane]);
+    }
+  } else {
+    float lqz[kMaxK], amax = -INFINITY;
+#pragma unroll
+    for (int z = 0; z < kMaxK; ++z) {
+      lqz[z] = 0.f;
+      if (z < K) {
+        if (act) {
+          const int q = ell + z * ell + lane;
+          lqz[z] = (in.xg[q] - in.m[q]) * invT - logf(in.s[q]);
+        }
+        float v = __shfl_up_sync(0xffffffffu, lqz[z], 1);
+        if (lane == 0) v = 0.f;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const float t = __shfl_up_sync(0xffffffffu, v, o);
+          if (lane >= o) v += t;
+        }
+        lpi[z] = (mix_w ? logf(mix_w[z]) : 0.f) + v;
+        amax = fmaxf(amax, lpi[z]);
+      }
+    }
+    float sa = 0.f;
+#pragma unroll
+    for (int z = 0; z < kMaxK; ++z)
+      if (z < K) sa += expf(lpi[z] - amax);
+    const float norm = amax + logf(sa);
+    float tmax = -INFINITY;
+#pragma unroll
+    for (int z = 0; z < kMaxK; ++z) {
+      if (z < K) {
+        lpi[z] -= norm;
+        tmax = fmaxf(tmax, lpi[z] + lqz[z]);
+      }
+    }
+    float st = 0.f;
+#pragma unroll
+    for (int z = 0; z < kMaxK; ++z)
+      if (z < K) st += expf(lpi[z] + lqz[z] - tmax);
+    const float lq = tmax + logf(st);
+    const float lp = act ? (in.xg[lane] - in.m[lane]) * invT - logf(in.s[lane]) : 0.f;
+    rho = expf(lp - lq);
+    finite = isfinite(norm) && isfinite(lp) && isfinite(lq);
+  }
+  const float thr = fminf(1.f, rho);
+  const float band = K == 1 ? 1e-5f : 2e-4f;
+  const bool close = act && (!finite || isnan(rho) || fabsf(uu - thr) < band);
+  if (__any_sync(0xffffffffu, close)) return decide_warp_fp64(in, u, mix_w);
+  const unsigned stop = __ballot_sync(0xffffffffu, act && !(uu < thr));
+  DecideOut o;
+  o.j = stop ? __ffs(stop) - 1 : ell;
+  o.bad = 0;
+  o.ct = o.mt = 0.f;
+  const int src = o.j & 31;
+  float lpj[kMaxK];
+#pragma unroll
+  for (int z = 0; z < kMaxK; ++z) lpj[z] = __shfl_sync(0xffffffffu, lpi[z], src);
+  if (o.j < ell) {
+    o.ct = 1.f / in.s[o.j];
+    o.mt = in.m[o.j];
+#pragma unroll
+    for (int z = 0; z < kMaxK; ++z) {
+      if (z < K) {
+        const int q = ell + z * ell + o.j;
+        o.cz[z] = expf(lpj[z]) / in.s[q];
+        o.mz[z] = in.m[q];
+      } else {
+        o.cz[z] = 0.f;
+        o.mz[z] = 0.f;
+      }
+    }
+  }
+  return o;
+}
+
+__device__ __forceinline__ DecideOut decide_warp_fp64(const DecideIn& in, const float* u, const float* mix_w) {
   const int lane = threadIdx.x & 31;
   const int ell = in.ell, K = in.K;
   const double T = static_cast<double>(in.T);

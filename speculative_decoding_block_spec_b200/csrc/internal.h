@@ -80,15 +80,13 @@ struct FusedArgs {
   int32_t* accept_len;
   int32_t* out_tokens;
   int* status;
-  int* ctl;                 // [0] epoch, [1] work counter, [2] exit counter
-  int* req_cnt;             // [B] statistics chunks done, reset by the decider
-  int* tterm;               // [B] terminal chunks done, reset by the last one
+  int* ctl;                 // [0] epoch, [2] exit counter
+  unsigned long long* req_units;  // [B] window units streamed, reset by the decider
+  unsigned long long* keys;  // [2B] best residual / bonus key per request, cleared by the last block
   int* dready;              // [B] epoch + 1 once the decision is published
   Decision* dec;            // [B]
-  TermPart* tpart;          // [B * Pt]
   float* xg;                // [rows] logit at the drafted token
-  float2* part;             // [rows * cpr] statistics partials
-  int cpr;                  // statistics chunks per row
+  float2* part;             // [grid + rows] statistics partials, slot block + row
   int64_t Vu;               // 16-byte units per row
   int Pt;                   // terminal chunks per request
   int64_t Vq;               // 8-element groups per row
@@ -97,9 +95,8 @@ struct FusedArgs {
 // Fused-path geometry (host and device agree on these).
 constexpr int kFusedStageBytes = 32768;
 constexpr int kFusedStages = 6;
-constexpr int kFusedMaxB = 512;
+constexpr int kFusedMaxB = 1024;
 constexpr int kFusedPtMax = 192;
-int fused_cpr(int64_t V, int dtype);
 int fused_pt(int64_t V, int dtype, int K);
 size_t fused_smem_bytes(int B);
 cudaError_t launch_fused(const FusedArgs& a, int dtype, int grid, cudaStream_t st);

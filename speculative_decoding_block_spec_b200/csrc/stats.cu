@@ -116,6 +116,7 @@ __device__ __forceinline__ void merge_row(const float2* part, int64_t r, int64_t
   m = -INFINITY;
   s = 0.f;
   for (int64_t c = c0; c <= c1; ++c) {
+    if (split_start(c + 1, N, G) == split_start(c, N, G)) continue;  // empty share (N < grid): no partial
     const float2 p = part[c + r];
     ms_merge(m, s, p.x, p.y, k);
   }

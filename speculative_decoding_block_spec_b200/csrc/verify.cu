@@ -117,6 +117,7 @@ __global__ void __launch_bounds__(kThreads) k_accept_sample(VerifyArgs a, float 
     const int64_t c0 = split_owner(r * a.Vu, N, a.G), c1 = split_owner((r + 1) * a.Vu - 1, N, a.G);
     float m = -INFINITY, s = 0.f;
     for (int64_t c = c0; c <= c1; ++c) {
+      if (split_start(c + 1, N, a.G) == split_start(c, N, a.G)) continue;  // empty share: no partial
       const float2 pr = a.rpart[c + r];
       ms_merge(m, s, pr.x, pr.y, k);
     }
