@@ -66,12 +66,12 @@ typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
 #define SPEC_DEV_NONFINITE 2    /* a needed row had a non-finite max or normaliser: accept_len = -1 */
 #define SPEC_DEV_VERIFY_LEN 4   /* verify_len[b] outside [0, L]: accept_len = -1 */
 #define SPEC_DEV_SCORES 8       /* a survival score outside [0, 1] or NaN */
-#define SPEC_DEV_TIMEOUT 16     /* an internal wait ran out (1 s); the call's outputs are not valid */
 
 /* Limits. */
 #define SPEC_MAX_L 32
 #define SPEC_MAX_K 8
 #define SPEC_MAX_B 4096
+#define SPEC_MAX_V 1048576      /* vocabulary of the verify calls (terminal token packed in 20 bits) */
 #define SPEC_MAX_DVL_ELEMS 16384 /* B * L for dvl_allocate_pack */
 
 /* Human-readable name of a spec_status value. Host only; never fails. */
@@ -135,14 +135,9 @@ int spec_softmax_T(const void* logits, int dtype, int64_t rows, int64_t V, int64
  *   accept_len     [B] int32 out: j (number of accepted draft tokens).
  *   out_tokens     [B, L+1] int32 out: x_0..x_{j-1}, terminal token, then -1.
  *   workspace      >= spec_verify_workspace_size(B, L, 1, V) bytes, zeroed once.
- * Limits: 1 <= B <= SPEC_MAX_B, 0 <= L <= SPEC_MAX_L, V >= 1.
- * Execution: with 16-byte-aligned logits and noise, V a multiple of 8 and
- * B <= 512 the whole call is one persistent kernel (one block per SM) that
- * streams the window through shared memory with bulk copies, takes each
- * request's decision as soon as its rows are done and draws its terminal
- * token while later requests still stream; otherwise it is the two stages
- * of spec_verify_window_stats + spec_verify_accept. Both give the same
- * decisions (bit-identical outputs away from the 1e-6 margins).
+ * Limits: 1 <= B <= SPEC_MAX_B, 0 <= L <= SPEC_MAX_L, 1 <= V <= SPEC_MAX_V.
+ * Execution: the two stages of spec_verify_window_stats and
+ * spec_verify_accept, chained with programmatic dependent launch.
  */
 int spec_verify_block(const void* target_logits, const int32_t* target_row_off,
                       const void* draft_logits, int dtype,
@@ -184,9 +179,10 @@ int spec_verify_mixture(const void* target_logits, const int32_t* target_row_off
  * verify window ([DBLAST] "What would settle it"; same T for target and
  * draft): for every request b, target rows 0..l_b-1 and the K draft rows of
  * positions 0..l_b-1 (l_b = verify_len[b], L if NULL) are streamed once and
- * their (max, normaliser) statistics are written into the workspace. Target
- * row l_b (the bonus row) needs no normaliser and is not read here. With
- * L == 0 nothing is launched; draft_logits may then be NULL.
+ * their (max, normaliser) statistics, and each row's logit at the drafted
+ * token, are written into the workspace. Target row l_b (the bonus row)
+ * needs no normaliser and is not read here. With L == 0 nothing is launched;
+ * draft_logits and draft_tokens may then be NULL.
  *
  * spec_verify_accept — stage 2: category posterior (K > 1), accept tests,
  * first rejection, residual / bonus Gumbel-max draw and outputs, exactly as
@@ -197,7 +193,8 @@ int spec_verify_mixture(const void* target_logits, const int32_t* target_row_off
  * Arguments and limits as spec_verify_mixture.
  */
 int spec_verify_window_stats(const void* target_logits, const int32_t* target_row_off,
-                             const void* draft_logits, int K, int dtype, const int32_t* verify_len,
+                             const void* draft_logits, int K, int dtype,
+                             const int32_t* draft_tokens, const int32_t* verify_len,
                              int B, int L, int64_t V, float T,
                              void* workspace, size_t ws_bytes, spec_stream_t stream);
 

@@ -22,11 +22,11 @@ import torch
 __all__ = ["SpecError", "Workspace", "lib", "softmax_T", "spec_softmax_T", "spec_verify_block",
            "spec_verify_mixture", "spec_verify_window_stats", "spec_verify_accept", "dvl_allocate_pack", "verify_workspace_size", "softmax_workspace_size",
            "dvl_workspace_size", "LIB_PATH", "EXPORTS", "DEV_TOKEN_RANGE", "DEV_NONFINITE", "DEV_VERIFY_LEN",
-           "DEV_SCORES", "DEV_TIMEOUT"]
+           "DEV_SCORES"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libspecv.so")
 
-DEV_TOKEN_RANGE, DEV_NONFINITE, DEV_VERIFY_LEN, DEV_SCORES, DEV_TIMEOUT = 1, 2, 4, 8, 16
+DEV_TOKEN_RANGE, DEV_NONFINITE, DEV_VERIFY_LEN, DEV_SCORES = 1, 2, 4, 8
 _F32, _BF16 = 0, 1
 
 _P, _I, _I64, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
@@ -39,7 +39,7 @@ _SIGS = {
     "spec_softmax_T": ([_P, _I, _I64, _I64, _I64, _F, _P, _P, _P, _P, _SZ, _P], _I),
     "spec_verify_block": ([_P, _P, _P, _I, _P, _P, _P, _P, _I, _I, _I64, _F, _P, _P, _P, _SZ, _P], _I),
     "spec_verify_mixture": ([_P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _I, _I, _I64, _F, _P, _P, _P, _SZ, _P], _I),
-    "spec_verify_window_stats": ([_P, _P, _P, _I, _I, _P, _I, _I, _I64, _F, _P, _SZ, _P], _I),
+    "spec_verify_window_stats": ([_P, _P, _P, _I, _I, _P, _P, _I, _I, _I64, _F, _P, _SZ, _P], _I),
     "spec_verify_accept": ([_P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _I, _I, _I64, _F, _P, _P, _P, _SZ, _P], _I),
     "dvl_allocate_pack": ([_P, _I, _I, _I, _P, _P, _P, _P, _P, _I, _I64, _P, _SZ, _P], _I),
 }
@@ -206,15 +206,17 @@ def spec_verify_mixture(target, draft, mix_w, tokens, u, g, T, *, verify_len=Non
     return acc, outt
 
 
-def spec_verify_window_stats(target, draft, T, workspace, *, K=1, L=None, verify_len=None, target_row_off=None):
+def spec_verify_window_stats(target, draft, tokens, T, workspace, *, verify_len=None, target_row_off=None):
     """Stage 1 of verification: temperature-softmax statistics of the verify
-    window into `workspace` (draft [B, L, V] for K == 1, else [B, K, L, V])."""
-    B = target.shape[0] if target_row_off is None else target_row_off.shape[0]
-    L = draft.shape[-2] if L is None else L
+    window, and each row's logit at the drafted token, into `workspace`
+    (draft [B, L, V] for K == 1, else [B, K, L, V]; tokens [B, L] int32)."""
+    B, L = tokens.shape
+    K = 1 if draft.dim() == 3 else draft.shape[1]
     V = draft.shape[-1]
     _call("spec_verify_window_stats", _dev(target, "target"), _opt(target_row_off, "target_row_off", torch.int32),
-          _dev(draft, "draft"), K, _dtype_code(draft), _opt(verify_len, "verify_len", torch.int32), B, L, V,
-          float(T), workspace.ptr(), workspace.nbytes, _stream(draft))
+          _dev(draft, "draft"), K, _dtype_code(draft), _dev(tokens, "tokens", torch.int32),
+          _opt(verify_len, "verify_len", torch.int32), B, L, V, float(T), workspace.ptr(), workspace.nbytes,
+          _stream(draft))
 
 
 def spec_verify_accept(target, draft, tokens, u, g, T, workspace, *, mix_w=None, verify_len=None,

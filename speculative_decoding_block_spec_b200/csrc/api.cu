@@ -34,34 +34,23 @@ int sm_count() {
   return sms;
 }
 
-// Verify workspace: persistent state first (never overlapped), then scratch
-// that the fused and the two-stage paths share.
+// Verify workspace: persistent state first (zero between calls), then scratch.
 struct VerifyLayout {
-  size_t ctl, req_units, keys, dready, tickets;      // persistent counters and flags
-  size_t tpart, rpart;                               // two-stage scratch
-  size_t dec, tpart_f, xg, part_f;                   // fused scratch
+  size_t ticket, keys;     // persistent: sampling-grid ticket, terminal keys [2B]
+  size_t dec, xg, rpart;   // scratch
   size_t total;
 };
 
 VerifyLayout verify_layout(int B, int L, int K, int64_t V) {
+  (void)V;
   VerifyLayout l;
-  const size_t b4 = align256(static_cast<size_t>(B) * sizeof(int));
-  l.ctl = kHeader;
-  l.req_units = l.ctl + 256;
-  l.keys = l.req_units + align256(static_cast<size_t>(B) * sizeof(unsigned long long));
-  l.dready = l.keys + align256(static_cast<size_t>(2 * B) * sizeof(unsigned long long));
-  l.tickets = l.dready + b4;
-  const size_t scratch = l.tickets + b4;
   const size_t rows = static_cast<size_t>(B) * (K + 1) * L;
-  l.tpart = scratch;
-  l.rpart = l.tpart + align256(static_cast<size_t>(B) * kPMax * sizeof(TermPart));
-  const size_t split_end = l.rpart + align256((static_cast<size_t>(kGMax) + rows) * sizeof(float2));
-  l.dec = scratch;
-  l.tpart_f = l.dec + align256(static_cast<size_t>(B) * sizeof(Decision));
-  l.xg = l.tpart_f + align256(static_cast<size_t>(B) * kFusedPtMax * sizeof(TermPart));
-  l.part_f = l.xg + align256(rows * sizeof(float));
-  const size_t fused_end = l.part_f + align256((static_cast<size_t>(kGMax) + rows) * 16 * sizeof(float2));
-  l.total = std::max(split_end, fused_end);
+  l.ticket = kHeader;
+  l.keys = l.ticket + 256;
+  l.dec = l.keys + align256(static_cast<size_t>(2 * B) * sizeof(unsigned long long));
+  l.xg = l.dec + align256(static_cast<size_t>(B) * sizeof(Decision));
+  l.rpart = l.xg + align256(rows * sizeof(float));
+  l.total = l.rpart + align256((static_cast<size_t>(kGMax) + rows) * sizeof(float2));
   return l;
 }
 
@@ -77,9 +66,9 @@ int verify_check(const void* target, const int32_t* row_off, const void* draft, 
   // [B, L] and [B, K, L, V] arrays are empty when L == 0, so their pointers may then be NULL.
   if (!target || (L > 0 && !draft)) return SPEC_ERR_ARG;
   if (accept_stage && (!g || !accept_len || !out_tokens || (L > 0 && (!tokens || !u)))) return SPEC_ERR_ARG;
-  if (!dtype_ok(dtype) || V < 1 || V > 0x7fffffffLL || !(T > 0.f) || !std::isfinite(T)) return SPEC_ERR_ARG;
+  if (!dtype_ok(dtype) || V < 1 || !(T > 0.f) || !std::isfinite(T)) return SPEC_ERR_ARG;
   if (B < 1 || L < 0 || K < 1) return SPEC_ERR_ARG;
-  if (!verify_shape_ok(B, L, K)) return SPEC_ERR_UNSUPPORTED;
+  if (!verify_shape_ok(B, L, K) || V > SPEC_MAX_V) return SPEC_ERR_UNSUPPORTED;
   if (accept_stage && K > 1 && !mix_w) return SPEC_ERR_ARG;
   if (!ws) return SPEC_ERR_WORKSPACE;
   if (ws_bytes < verify_layout(B, L, K, V).total) return SPEC_ERR_WORKSPACE;
@@ -98,7 +87,8 @@ bool stats_vec(const void* target, const void* draft, int dtype, int64_t V) {
 }
 
 int launch_stats_stage(const void* target, const int32_t* row_off, const void* draft, int K, int dtype,
-                       const int32_t* vlen, int B, int L, int64_t V, float T, void* ws, cudaStream_t st) {
+                       const int32_t* tokens, const int32_t* vlen, int B, int L, int64_t V, float T, void* ws,
+                       cudaStream_t st) {
   if (L == 0) return SPEC_OK;
   const bool vec = stats_vec(target, draft, dtype, V);
   const VerifyLayout lay = verify_layout(B, L, K, V);
@@ -107,6 +97,8 @@ int launch_stats_stage(const void* target, const int32_t* row_off, const void* d
   rs.draft = draft;
   rs.row_off = row_off;
   rs.vlen = vlen;
+  rs.tokens = tokens;
+  rs.xg = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.xg);
   rs.stride = V;
   rs.rows = 0;
   rs.B = B;
@@ -142,8 +134,10 @@ int launch_accept_stage(const void* target, const int32_t* row_off, const void* 
   a.accept_len = accept_len;
   a.out_tokens = out_tokens;
   a.status = reinterpret_cast<int*>(w);
-  a.tickets = reinterpret_cast<int*>(w + lay.tickets);
-  a.tpart = reinterpret_cast<TermPart*>(w + lay.tpart);
+  a.tickets = reinterpret_cast<int*>(w + lay.ticket);
+  a.keys = reinterpret_cast<unsigned long long*>(w + lay.keys);
+  a.dec = reinterpret_cast<Decision*>(w + lay.dec);
+  a.xg = reinterpret_cast<const float*>(w + lay.xg);
   a.rpart = reinterpret_cast<const float2*>(w + lay.rpart);
   a.Vu = units_per_row(V, dtype, vec);
   a.G = stats_grid(dtype, vec, static_cast<int64_t>(B) * (K + 1) * L * a.Vu);
@@ -155,51 +149,6 @@ int launch_accept_stage(const void* target, const int32_t* row_off, const void* 
   return map_cuda(launch_accept_sample(a, dtype, vec_term, st));
 }
 
-// The one-kernel path needs the vector path for every operand, V a multiple
-// of 8 and a terminal split that fits its stage ring.
-bool fused_ok(const void* target, const void* draft, const float* g, int dtype, int B, int L, int K, int64_t V) {
-  return L >= 1 && B <= kFusedMaxB && V % 8 == 0 && V <= (1 << 20) && stats_vec(target, draft, dtype, V) &&
-         aligned(g, 16) &&
-         fused_pt(V, dtype, K) <= kFusedPtMax;
-}
-
-int launch_fused_stage(const void* target, const int32_t* row_off, const void* draft, const float* mix_w, int K,
-                       int dtype, const int32_t* tokens, const int32_t* vlen, const float* u, const float* g, int B,
-                       int L, int64_t V, float T, int32_t* accept_len, int32_t* out_tokens, void* ws,
-                       cudaStream_t st) {
-  const VerifyLayout lay = verify_layout(B, L, K, V);
-  char* w = static_cast<char*>(ws);
-  FusedArgs a = {};
-  a.target = target;
-  a.row_off = row_off;
-  a.draft = draft;
-  a.mix_w = mix_w;
-  a.tokens = tokens;
-  a.vlen = vlen;
-  a.u = u;
-  a.g = g;
-  a.B = B;
-  a.L = L;
-  a.K = K;
-  a.V = V;
-  a.T = T;
-  a.k = static_cast<float>(1.4426950408889634 / static_cast<double>(T));
-  a.accept_len = accept_len;
-  a.out_tokens = out_tokens;
-  a.status = reinterpret_cast<int*>(w);
-  a.ctl = reinterpret_cast<int*>(w + lay.ctl);
-  a.req_units = reinterpret_cast<unsigned long long*>(w + lay.req_units);
-  a.keys = reinterpret_cast<unsigned long long*>(w + lay.keys);
-  a.dready = reinterpret_cast<int*>(w + lay.dready);
-  a.dec = reinterpret_cast<Decision*>(w + lay.dec);
-  a.xg = reinterpret_cast<float*>(w + lay.xg);
-  a.part = reinterpret_cast<float2*>(w + lay.part_f);
-  a.Vu = units_per_row(V, dtype, true);
-  a.Pt = fused_pt(V, dtype, K);
-  a.Vq = V / 8;
-  return map_cuda(launch_fused(a, dtype, sm_count(), st));
-}
-
 int verify_common(const void* target, const int32_t* row_off, const void* draft, const float* mix_w, int K,
                   int dtype, const int32_t* tokens, const int32_t* vlen, const float* u, const float* g, int B,
                   int L, int64_t V, float T, int32_t* accept_len, int32_t* out_tokens, void* ws, size_t ws_bytes,
@@ -207,10 +156,7 @@ int verify_common(const void* target, const int32_t* row_off, const void* draft,
   int e = verify_check(target, row_off, draft, mix_w, K, dtype, tokens, vlen, u, g, B, L, V, T, accept_len,
                        out_tokens, ws, ws_bytes, true);
   if (e) return e;
-  if (fused_ok(target, draft, g, dtype, B, L, K, V))
-    return launch_fused_stage(target, row_off, draft, mix_w, K, dtype, tokens, vlen, u, g, B, L, V, T, accept_len,
-                              out_tokens, ws, st);
-  e = launch_stats_stage(target, row_off, draft, K, dtype, vlen, B, L, V, T, ws, st);
+  e = launch_stats_stage(target, row_off, draft, K, dtype, tokens, vlen, B, L, V, T, ws, st);
   if (e) return e;
   return launch_accept_stage(target, row_off, draft, mix_w, K, dtype, tokens, vlen, u, g, B, L, V, T, accept_len,
                              out_tokens, ws, st);
@@ -237,7 +183,7 @@ size_t spec_softmax_workspace_size(int64_t rows) {
 }
 
 size_t spec_verify_workspace_size(int B, int L, int K, int64_t V) {
-  if (!verify_shape_ok(B, L, K) || V < 1 || V > 0x7fffffffLL) return 0;
+  if (!verify_shape_ok(B, L, K) || V < 1 || V > SPEC_MAX_V) return 0;
   return verify_layout(B, L, K, V).total;
 }
 
@@ -304,13 +250,14 @@ int spec_verify_mixture(const void* target_logits, const int32_t* target_row_off
 }
 
 int spec_verify_window_stats(const void* target_logits, const int32_t* target_row_off, const void* draft_logits,
-                             int K, int dtype, const int32_t* verify_len, int B, int L, int64_t V, float T,
-                             void* workspace, size_t ws_bytes, spec_stream_t stream) {
-  const int e = verify_check(target_logits, target_row_off, draft_logits, nullptr, K, dtype, nullptr, verify_len,
+                             int K, int dtype, const int32_t* draft_tokens, const int32_t* verify_len, int B, int L,
+                             int64_t V, float T, void* workspace, size_t ws_bytes, spec_stream_t stream) {
+  if (L > 0 && !draft_tokens) return SPEC_ERR_ARG;
+  const int e = verify_check(target_logits, target_row_off, draft_logits, nullptr, K, dtype, draft_tokens, verify_len,
                              nullptr, nullptr, B, L, V, T, nullptr, nullptr, workspace, ws_bytes, false);
   if (e) return e;
-  return launch_stats_stage(target_logits, target_row_off, draft_logits, K, dtype, verify_len, B, L, V, T, workspace,
-                            reinterpret_cast<cudaStream_t>(stream));
+  return launch_stats_stage(target_logits, target_row_off, draft_logits, K, dtype, draft_tokens, verify_len, B, L, V, T,
+                            workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int spec_verify_accept(const void* target_logits, const int32_t* target_row_off, const void* draft_logits,

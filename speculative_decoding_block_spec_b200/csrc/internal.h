@@ -17,22 +17,20 @@ struct RowSpace {
   const void* draft;
   const int32_t* row_off;
   const int32_t* vlen;
+  const int32_t* tokens;    // verify mode: drafted tokens [B, L]
+  float* xg;                // verify mode: out, logit at the drafted token of each window row
   int64_t stride;
   int64_t rows;
   int B, L, K;
   int verify;
 };
 
-// Per-request terminal-draw partial of one sampling block.
-struct TermPart {
-  double res_score;  // best residual score (ln r + g), -inf if none
-  double bon_score;  // best bonus-rule score (x / T + g)
-  int res_idx;       // its token, -1 if none
-  int bon_idx;
-  int pad[2];
+// Per-request decision, written by block 0 of the request in the sampling kernel.
+struct Decision {
+  int j, flags;
 };
 
-// Everything the accept/sample kernel reads.
+// Everything the accept/sample kernel reads and writes.
 struct VerifyArgs {
   const void* target;
   const int32_t* row_off;
@@ -48,58 +46,15 @@ struct VerifyArgs {
   int32_t* accept_len;
   int32_t* out_tokens;
   int* status;
-  int* tickets;             // [B], self-resetting
-  TermPart* tpart;          // [B * P]
+  int* tickets;             // [1] blocks finished, reset by the last one
+  unsigned long long* keys; // [2B] best residual / bonus key per request, cleared by the last block
+  Decision* dec;            // [B]
+  const float* xg;          // [rows] logit at the drafted token (from the statistics kernel)
   const float2* rpart;      // row-statistics partials
   int G;                    // row-statistics grid size
   int64_t Vu;               // row-statistics units per row
   int P;                    // sampling blocks per request
 };
-
-// Per-request decision published by the fused kernel's decider block.
-struct Decision {
-  int j, flags, ell, pad;
-  float ct, mt, pad2[2];
-  float cz[8], mz[8];
-};
-
-// Everything the fused verify kernel reads and writes.
-struct FusedArgs {
-  const void* target;
-  const int32_t* row_off;
-  const void* draft;
-  const float* mix_w;
-  const int32_t* tokens;
-  const int32_t* vlen;
-  const float* u;
-  const float* g;
-  int B, L, K;
-  int64_t V;
-  float T;
-  float k;                  // log2(e) / T
-  int32_t* accept_len;
-  int32_t* out_tokens;
-  int* status;
-  int* ctl;                 // [0] epoch, [2] exit counter
-  unsigned long long* req_units;  // [B] window units streamed, reset by the decider
-  unsigned long long* keys;  // [2B] best residual / bonus key per request, cleared by the last block
-  int* dready;              // [B] epoch + 1 once the decision is published
-  Decision* dec;            // [B]
-  float* xg;                // [rows] logit at the drafted token
-  float2* part;             // [grid + rows] statistics partials, slot block + row
-  int64_t Vu;               // 16-byte units per row
-  int Pt;                   // terminal chunks per request
-  int64_t Vq;               // 8-element groups per row
-};
-
-// Fused-path geometry (host and device agree on these).
-constexpr int kFusedStageBytes = 32768;
-constexpr int kFusedStages = 6;
-constexpr int kFusedMaxB = 1024;
-constexpr int kFusedPtMax = 192;
-int fused_pt(int64_t V, int dtype, int K);
-size_t fused_smem_bytes(int B);
-cudaError_t launch_fused(const FusedArgs& a, int dtype, int grid, cudaStream_t st);
 
 // Units of work per row: 16-byte vectors on the vector path, else elements.
 inline int64_t units_per_row(int64_t V, int dtype, bool vec) {

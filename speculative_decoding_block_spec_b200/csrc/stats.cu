@@ -24,9 +24,12 @@ namespace specv {
 
 constexpr int kUnroll = 4;  // 16-byte vectors in flight per thread per group
 
+// Row r of the walk; in verify mode also the drafted token of its position
+// (column of the logit to record), -1 if none or out of range.
 template <int DT>
-__device__ __forceinline__ const char* row_pointer(const RowSpace& rs, int64_t r, const int* rowoff) {
+__device__ __forceinline__ const char* row_pointer(const RowSpace& rs, int64_t r, const int* rowoff, int& tok) {
   constexpr int64_t esz = Elem<DT>::kBytes;
+  tok = -1;
   if (!rs.verify) return static_cast<const char*>(rs.target) + r * rs.stride * esz;
   int lo = 0, hi = rs.B - 1;  // last request whose first row is <= r
   while (lo < hi) {
@@ -37,6 +40,8 @@ __device__ __forceinline__ const char* row_pointer(const RowSpace& rs, int64_t r
   const int q = static_cast<int>(r - rowoff[b]);
   int l = rs.vlen ? rs.vlen[b] : rs.L;
   if (l < 0 || l > rs.L) l = 0;
+  const int x = __ldg(rs.tokens + static_cast<int64_t>(b) * rs.L + (q < l ? q : (q - l) % l));
+  tok = (x >= 0 && x < rs.stride) ? x : -1;
   if (q < l) {
     const int64_t base = rs.row_off ? static_cast<int64_t>(rs.row_off[b]) : static_cast<int64_t>(b) * (rs.L + 1);
     return static_cast<const char*>(rs.target) + (base + q) * rs.stride * esz;
@@ -46,10 +51,14 @@ __device__ __forceinline__ const char* row_pointer(const RowSpace& rs, int64_t r
          ((static_cast<int64_t>(b) * rs.K + z) * rs.L + i) * rs.stride * esz;
 }
 
-// Per-thread statistics of units [u0, u1) of one row.
+// Per-thread statistics of units [u0, u1) of one row; the thread that meets
+// element `tok` of the row records its logit in *xg.
 template <int DT, bool VEC>
 __device__ __forceinline__ void segment_stats(const char* row, int64_t u0, int64_t u1, float k, float& m,
-                                              float& s) {
+                                              float& s, int tok, float* xg) {
+  constexpr int E = VEC ? Elem<DT>::kPerVec : 1;
+  if (tok >= 0 && tok / E >= u0 && tok / E < u1 && (tok / E - u0) % kThreads == threadIdx.x)
+    *xg = Elem<DT>::at(row, tok);
   int64_t u = u0 + threadIdx.x;
   if constexpr (VEC) {
     const uint4* rv = reinterpret_cast<const uint4*>(row);
@@ -100,9 +109,10 @@ __global__ void __launch_bounds__(kThreads) k_row_stats(RowSpace rs, int64_t Vu,
   for (int64_t e = split_start(blockIdx.x, N, G); e < e1;) {
     const int64_t r = e / Vu;
     const int64_t se = min(e1, (r + 1) * Vu);
-    const char* row = row_pointer<DT>(rs, r, rowoff);
+    int tok;
+    const char* row = row_pointer<DT>(rs, r, rowoff, tok);
     float m = -INFINITY, s = 0.f;
-    segment_stats<DT, VEC>(row, e - r * Vu, se - r * Vu, k, m, s);
+    segment_stats<DT, VEC>(row, e - r * Vu, se - r * Vu, k, m, s, tok, rs.xg ? rs.xg + r : nullptr);
     block_merge(m, s, k, red);
     if (threadIdx.x == 0) part[blockIdx.x + r] = make_float2(m, s);
     e = se;

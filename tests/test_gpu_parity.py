@@ -74,7 +74,7 @@ def _verify(d, x, T, verify_len=None, target=None, row_off=None, path="fused"):
     if path == "split":
         B, L = d["tokens"].shape
         ws = specv.Workspace(specv.verify_workspace_size(B, L, x.w.K, x.w.V))
-        specv.spec_verify_window_stats(tgt, d["draft"], T, ws, K=x.w.K, L=L, verify_len=verify_len,
+        specv.spec_verify_window_stats(tgt, d["draft"], d["tokens"], T, ws, verify_len=verify_len,
                                        target_row_off=row_off)
         return specv.spec_verify_accept(tgt, d["draft"], d["tokens"], d["u"], d["g"], T, ws, mix_w=mix,
                                         verify_len=verify_len, target_row_off=row_off)
@@ -215,7 +215,7 @@ def test_device_flags_and_isolation(path):
     ws = specv.Workspace(specv.verify_workspace_size(4, 8, 2, 4096))
     if path == "split":
         vlt = torch.from_numpy(vl).cuda()
-        specv.spec_verify_window_stats(d["target"], d["draft"], 1.0, ws, K=2, verify_len=vlt)
+        specv.spec_verify_window_stats(d["target"], d["draft"], d["tokens"], 1.0, ws, verify_len=vlt)
         acc, out = specv.spec_verify_accept(d["target"], d["draft"], d["tokens"], d["u"], d["g"], 1.0, ws,
                                             mix_w=d["mix_w"], verify_len=vlt)
     else:
@@ -244,7 +244,7 @@ def test_workspace_reuse_is_self_resetting():
     first = [t.clone() for t in first]
     for it in range(6):
         if it % 3 == 2:
-            specv.spec_verify_window_stats(d["target"], d["draft"], 1.0, ws)
+            specv.spec_verify_window_stats(d["target"], d["draft"], d["tokens"], 1.0, ws)
             again = specv.spec_verify_accept(d["target"], d["draft"], d["tokens"], d["u"], d["g"], 1.0, ws)
         else:
             again = specv.spec_verify_block(d["target"], d["draft"], d["tokens"], d["u"], d["g"], 1.0,
