@@ -73,6 +73,7 @@ typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
 #define SPEC_MAX_B 4096
 #define SPEC_MAX_V 1048576      /* vocabulary of the verify calls (terminal token packed in 20 bits) */
 #define SPEC_MAX_DVL_ELEMS 16384 /* B * L for dvl_allocate_pack */
+#define SPEC_NOALLOC_MAX_ROWS 4096 /* rows of spec_softmax_T_noalloc (fixed 48 KiB scratch) */
 
 /* Human-readable name of a spec_status value. Host only; never fails. */
 const char* spec_status_string(int status);
@@ -104,6 +105,30 @@ int spec_workspace_init(void* workspace, size_t ws_bytes, spec_stream_t stream);
 int spec_softmax_T(const void* logits, int dtype, int64_t rows, int64_t V, int64_t row_stride,
                    float T, float* row_max, float* row_lse, float* probs,
                    void* workspace, size_t ws_bytes, spec_stream_t stream);
+
+/*
+ * spec_softmax_T_noalloc — spec_softmax_T for callers that cannot allocate
+ * device memory. The paper has no counterpart: this entry point exists only
+ * for such callers. Arguments, results and numerics are those of
+ * spec_softmax_T without the workspace; the call allocates nothing
+ * (no cudaMalloc, cudaFree or allocating library routine).
+ * Scratch: the statistics partials live in one fixed array inside the library
+ * (static __device__, 256-byte aligned, (2048 + SPEC_NOALLOC_MAX_ROWS) * 8
+ * bytes = 48 KiB on each device).
+ *   rows  0 <= rows <= SPEC_NOALLOC_MAX_ROWS; larger returns
+ *         SPEC_ERR_UNSUPPORTED before anything is launched.
+ * Set-up: the first call on a device looks up the array's device address with
+ * cudaGetSymbolAddress, with that device current (the current device must be
+ * the stream's device); a failed lookup returns SPEC_ERR_CUDA. Make that first
+ * call on each device before any stream capture begins.
+ * Sharing: every call on a device uses the same array. Nothing in it has to
+ * start at zero (each call writes every slot before it reads it), but calls
+ * whose kernels overlap on the GPU (different streams, or different host
+ * threads) race on the array and return wrong statistics: issue them in order
+ * on one stream.
+ */
+int spec_softmax_T_noalloc(const void* logits, int dtype, int64_t rows, int64_t V, int64_t row_stride,
+                           float T, float* row_max, float* row_lse, float* probs, spec_stream_t stream);
 
 /*
  * spec_verify_block — lossless speculative-sampling verification of B

@@ -19,7 +19,7 @@ import os
 
 import torch
 
-__all__ = ["SpecError", "Workspace", "lib", "softmax_T", "spec_softmax_T", "spec_verify_block",
+__all__ = ["SpecError", "Workspace", "lib", "softmax_T", "spec_softmax_T", "spec_softmax_T_noalloc", "NOALLOC_MAX_ROWS", "spec_verify_block",
            "spec_verify_mixture", "spec_verify_window_stats", "spec_verify_accept", "dvl_allocate_pack", "verify_workspace_size", "softmax_workspace_size",
            "dvl_workspace_size", "LIB_PATH", "EXPORTS", "DEV_TOKEN_RANGE", "DEV_NONFINITE", "DEV_VERIFY_LEN",
            "DEV_SCORES"]
@@ -27,6 +27,7 @@ __all__ = ["SpecError", "Workspace", "lib", "softmax_T", "spec_softmax_T", "spec
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libspecv.so")
 
 DEV_TOKEN_RANGE, DEV_NONFINITE, DEV_VERIFY_LEN, DEV_SCORES = 1, 2, 4, 8
+NOALLOC_MAX_ROWS = 4096  # SPEC_NOALLOC_MAX_ROWS
 _F32, _BF16 = 0, 1
 
 _P, _I, _I64, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
@@ -37,6 +38,7 @@ _SIGS = {
     "spec_dvl_workspace_size": ([_I], _SZ),
     "spec_workspace_init": ([_P, _SZ, _P], _I),
     "spec_softmax_T": ([_P, _I, _I64, _I64, _I64, _F, _P, _P, _P, _P, _SZ, _P], _I),
+    "spec_softmax_T_noalloc": ([_P, _I, _I64, _I64, _I64, _F, _P, _P, _P, _P], _I),
     "spec_verify_block": ([_P, _P, _P, _I, _P, _P, _P, _P, _I, _I, _I64, _F, _P, _P, _P, _SZ, _P], _I),
     "spec_verify_mixture": ([_P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _I, _I, _I64, _F, _P, _P, _P, _SZ, _P], _I),
     "spec_verify_window_stats": ([_P, _P, _P, _I, _I, _P, _P, _I, _I, _I64, _F, _P, _SZ, _P], _I),
@@ -148,6 +150,19 @@ def spec_softmax_T(logits, T, row_max, row_lse, probs=None, workspace=None):
           _dev(row_max, "row_max", torch.float32), _dev(row_lse, "row_lse", torch.float32),
           _opt(probs, "probs", torch.float32), ws.ptr(), ws.nbytes, _stream(logits))
     return ws
+
+
+def spec_softmax_T_noalloc(logits, T, row_max, row_lse, probs=None):
+    """C-ABI spec_softmax_T_noalloc on preallocated outputs: spec_softmax_T with
+    the library's fixed scratch instead of a workspace (rows <= NOALLOC_MAX_ROWS;
+    calls on one device must not overlap on the GPU)."""
+    rows, V = logits.shape
+    if rows > NOALLOC_MAX_ROWS:
+        raise ValueError("spec_softmax_T_noalloc: %d rows exceed the fixed scratch limit of %d rows"
+                         % (rows, NOALLOC_MAX_ROWS))
+    _call("spec_softmax_T_noalloc", _dev(logits, "logits"), _dtype_code(logits), rows, V, V, float(T),
+          _dev(row_max, "row_max", torch.float32), _dev(row_lse, "row_lse", torch.float32),
+          _opt(probs, "probs", torch.float32), _stream(logits))
 
 
 def softmax_T(logits, T, probs=False, workspace=None):

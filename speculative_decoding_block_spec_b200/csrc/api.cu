@@ -34,6 +34,29 @@ int sm_count() {
   return sms;
 }
 
+// Fixed scratch of spec_softmax_T_noalloc: the per-row statistics partials of
+// at most SPEC_NOALLOC_MAX_ROWS rows (kGMax + rows slots, as in the softmax
+// workspace after its header). Shared by every call on a device.
+static __device__ __align__(256) float2 g_noalloc_part[kGMax + SPEC_NOALLOC_MAX_ROWS];
+
+// Device address of g_noalloc_part on the current device, looked up once per
+// device (with that device current) and cached.
+int noalloc_scratch(float2** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SPEC_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return SPEC_ERR_UNSUPPORTED;
+  static std::mutex mu;
+  static void* cache[64] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_part) != cudaSuccess || !p) return SPEC_ERR_CUDA;
+    cache[dev] = p;
+  }
+  *out = static_cast<float2*>(cache[dev]);
+  return SPEC_OK;
+}
+
 // Verify workspace: persistent state first (zero between calls), then scratch.
 struct VerifyLayout {
   size_t ticket, keys;     // persistent: sampling-grid ticket, terminal keys [2B]
@@ -216,6 +239,36 @@ int spec_softmax_T(const void* logits, int dtype, int64_t rows, int64_t V, int64
                    (!probs || aligned(probs, 16));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   float2* part = reinterpret_cast<float2*>(static_cast<char*>(workspace) + kHeader);
+  const int64_t Vu = units_per_row(V, dtype, vec);
+  const int G = stats_grid(dtype, vec, rows * Vu);
+  RowSpace rs = {};
+  rs.target = logits;
+  rs.stride = row_stride;
+  rs.rows = rows;
+  rs.verify = 0;
+  int e = map_cuda(launch_row_stats(rs, dtype, vec, V, T, G, part, st));
+  if (e) return e;
+  return map_cuda(
+      launch_softmax_finalize(logits, dtype, vec, rows, V, row_stride, T, G, part, row_max, row_lse, probs, st));
+}
+
+int spec_softmax_T_noalloc(const void* logits, int dtype, int64_t rows, int64_t V, int64_t row_stride, float T,
+                           float* row_max, float* row_lse, float* probs, spec_stream_t stream) {
+  if (!logits || !row_max || !row_lse) return SPEC_ERR_ARG;
+  if (!dtype_ok(dtype) || rows < 0 || V < 1 || V > 0x7fffffffLL || row_stride < V || !(T > 0.f) ||
+      !std::isfinite(T))
+    return SPEC_ERR_ARG;
+  if (rows > SPEC_NOALLOC_MAX_ROWS) return SPEC_ERR_UNSUPPORTED;  // beyond the fixed scratch
+  const int es = esize(dtype);
+  if (!aligned(logits, es) || !aligned(row_max, 4) || !aligned(row_lse, 4) || (probs && !aligned(probs, 4)))
+    return SPEC_ERR_ARG;
+  if (rows == 0) return SPEC_OK;
+  float2* part = nullptr;
+  const int se = noalloc_scratch(&part);
+  if (se) return se;
+  const bool vec = (V * es) % 16 == 0 && (row_stride * es) % 16 == 0 && aligned(logits, 16) &&
+                   (!probs || aligned(probs, 16));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t Vu = units_per_row(V, dtype, vec);
   const int G = stats_grid(dtype, vec, rows * Vu);
   RowSpace rs = {};
