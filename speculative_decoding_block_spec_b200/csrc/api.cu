@@ -57,10 +57,22 @@ int noalloc_scratch(float2** out) {
   return SPEC_OK;
 }
 
+// Resident sampling blocks per SM (cached per device and variant).
+int accept_slots(int dtype, bool vec) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
+  static std::mutex mu;
+  static int cache[64][4] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  int& c = cache[dev][dtype * 2 + (vec ? 1 : 0)];
+  if (!c) c = accept_blocks_per_sm(dtype, vec);
+  return c;
+}
+
 // Verify workspace: persistent state first (zero between calls), then scratch.
 struct VerifyLayout {
-  size_t ticket, keys;     // persistent: sampling-grid ticket, terminal keys [2B]
-  size_t dec, xg, rpart;   // scratch
+  size_t ticket, keys;     // persistent: per-request tickets [B], terminal keys [2B]
+  size_t xg, rpart;        // scratch
   size_t total;
 };
 
@@ -69,9 +81,8 @@ VerifyLayout verify_layout(int B, int L, int K, int64_t V) {
   VerifyLayout l;
   const size_t rows = static_cast<size_t>(B) * (K + 1) * L;
   l.ticket = kHeader;
-  l.keys = l.ticket + 256;
-  l.dec = l.keys + align256(static_cast<size_t>(2 * B) * sizeof(unsigned long long));
-  l.xg = l.dec + align256(static_cast<size_t>(B) * sizeof(Decision));
+  l.keys = l.ticket + align256(static_cast<size_t>(B) * sizeof(int));
+  l.xg = l.keys + align256(static_cast<size_t>(2 * B) * sizeof(unsigned long long));
   l.rpart = l.xg + align256(rows * sizeof(float));
   l.total = l.rpart + align256((static_cast<size_t>(kGMax) + rows) * sizeof(float2));
   return l;
@@ -159,16 +170,16 @@ int launch_accept_stage(const void* target, const int32_t* row_off, const void* 
   a.status = reinterpret_cast<int*>(w);
   a.tickets = reinterpret_cast<int*>(w + lay.ticket);
   a.keys = reinterpret_cast<unsigned long long*>(w + lay.keys);
-  a.dec = reinterpret_cast<Decision*>(w + lay.dec);
   a.xg = reinterpret_cast<const float*>(w + lay.xg);
   a.rpart = reinterpret_cast<const float2*>(w + lay.rpart);
   a.Vu = units_per_row(V, dtype, vec);
   a.G = stats_grid(dtype, vec, static_cast<int64_t>(B) * (K + 1) * L * a.Vu);
-  // Blocks per request for the terminal row: about two waves over the SMs,
-  // at least 256 units of the row per block.
+  // Blocks per request for the terminal row: the whole (P, B) grid resident
+  // at once (no second wave), at least 256 units of the row per block.
   const int64_t term_units = vec_term ? V / (16 / esize(dtype)) : V;
-  const int64_t p_sm = (2 * static_cast<int64_t>(sm_count()) + B - 1) / B;
-  a.P = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({p_sm, kPMax, term_units / kThreads})));
+  const int64_t slots = static_cast<int64_t>(sm_count()) * accept_slots(dtype, vec_term);
+  const int64_t p_fit = std::max<int64_t>(1, slots / B);
+  a.P = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({p_fit, kPMax, term_units / kThreads})));
   return map_cuda(launch_accept_sample(a, dtype, vec_term, st));
 }
 

@@ -25,11 +25,6 @@ struct RowSpace {
   int verify;
 };
 
-// Per-request decision, written by block 0 of the request in the sampling kernel.
-struct Decision {
-  int j, flags;
-};
-
 // Everything the accept/sample kernel reads and writes.
 struct VerifyArgs {
   const void* target;
@@ -46,9 +41,8 @@ struct VerifyArgs {
   int32_t* accept_len;
   int32_t* out_tokens;
   int* status;
-  int* tickets;             // [1] blocks finished, reset by the last one
-  unsigned long long* keys; // [2B] best residual / bonus key per request, cleared by the last block
-  Decision* dec;            // [B]
+  int* tickets;             // [B] blocks of each request finished, reset by the request's last block
+  unsigned long long* keys; // [2B] best residual / bonus key per request, cleared by its last block
   const float* xg;          // [rows] logit at the drafted token (from the statistics kernel)
   const float2* rpart;      // row-statistics partials
   int G;                    // row-statistics grid size
@@ -72,6 +66,7 @@ cudaError_t launch_softmax_finalize(const void* logits, int dtype, bool vec, int
                                     float* row_lse, float* probs, cudaStream_t st);
 
 cudaError_t launch_accept_sample(const VerifyArgs& a, int dtype, bool vec, cudaStream_t st);
+int accept_blocks_per_sm(int dtype, bool vec);
 
 cudaError_t launch_dvl(const float* scores, int B, int L, int budget, int32_t* verify_len,
                        int32_t* offsets, int32_t* slot_map, int* status, int* ticket,

@@ -24,99 +24,164 @@ namespace specv {
 
 constexpr int kUnroll = 4;  // 16-byte vectors in flight per thread per group
 
-// Row r of the walk; in verify mode also the drafted token of its position
-// (column of the logit to record), -1 if none or out of range.
+// Geometry of the verify walk, built in shared memory by every block:
+// rowoff[b] first walk row of request b (rowoff[B] = total), base[b] target
+// row of its position 0. Request b owns (K+1)*l walk rows: l target rows,
+// then K draft categories of l rows each, l = verified length.
+struct Walk {
+  const int* rowoff;
+  const int* base;
+};
+
+// Row r of the walk and the address of the drafted token of its position
+// (nullptr outside verify mode). The token itself is loaded by the caller,
+// which uses it only after the row's first data has arrived.
 template <int DT>
-__device__ __forceinline__ const char* row_pointer(const RowSpace& rs, int64_t r, const int* rowoff, int& tok) {
+__device__ __forceinline__ const char* locate(const RowSpace& rs, const Walk& w, int64_t r, const int32_t*& tokp) {
   constexpr int64_t esz = Elem<DT>::kBytes;
-  tok = -1;
+  tokp = nullptr;
   if (!rs.verify) return static_cast<const char*>(rs.target) + r * rs.stride * esz;
   int lo = 0, hi = rs.B - 1;  // last request whose first row is <= r
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (rowoff[mid] <= r) lo = mid; else hi = mid - 1;
+    if (w.rowoff[mid] <= r) lo = mid; else hi = mid - 1;
   }
   const int b = lo;
-  const int q = static_cast<int>(r - rowoff[b]);
-  int l = rs.vlen ? rs.vlen[b] : rs.L;
-  if (l < 0 || l > rs.L) l = 0;
-  const int x = __ldg(rs.tokens + static_cast<int64_t>(b) * rs.L + (q < l ? q : (q - l) % l));
-  tok = (x >= 0 && x < rs.stride) ? x : -1;
+  const int q = static_cast<int>(r - w.rowoff[b]);
+  const int l = (w.rowoff[b + 1] - w.rowoff[b]) / (rs.K + 1);
   if (q < l) {
-    const int64_t base = rs.row_off ? static_cast<int64_t>(rs.row_off[b]) : static_cast<int64_t>(b) * (rs.L + 1);
-    return static_cast<const char*>(rs.target) + (base + q) * rs.stride * esz;
+    tokp = rs.tokens + static_cast<int64_t>(b) * rs.L + q;
+    return static_cast<const char*>(rs.target) + (static_cast<int64_t>(w.base[b]) + q) * rs.stride * esz;
   }
   const int q2 = q - l, z = q2 / l, i = q2 - z * l;
-  return static_cast<const char*>(rs.draft) +
-         ((static_cast<int64_t>(b) * rs.K + z) * rs.L + i) * rs.stride * esz;
+  tokp = rs.tokens + static_cast<int64_t>(b) * rs.L + i;
+  return static_cast<const char*>(rs.draft) + ((static_cast<int64_t>(b) * rs.K + z) * rs.L + i) * rs.stride * esz;
 }
 
-// Per-thread statistics of units [u0, u1) of one row; the thread that meets
-// element `tok` of the row records its logit in *xg.
-template <int DT, bool VEC>
-__device__ __forceinline__ void segment_stats(const char* row, int64_t u0, int64_t u1, float k, float& m,
-                                              float& s, int tok, float* xg) {
-  constexpr int E = VEC ? Elem<DT>::kPerVec : 1;
-  if (tok >= 0 && tok / E >= u0 && tok / E < u1 && (tok / E - u0) % kThreads == threadIdx.x)
-    *xg = Elem<DT>::at(row, tok);
-  int64_t u = u0 + threadIdx.x;
-  if constexpr (VEC) {
-    const uint4* rv = reinterpret_cast<const uint4*>(row);
+__device__ __forceinline__ int load_token(const int32_t* tokp) { return tokp ? __ldg(tokp) : -1; }
+
+// Element `idx` (0..E-1) of a 16-byte vector.
+template <int DT>
+__device__ __forceinline__ float vec_elem(const uint4& h, int idx) {
+  if constexpr (DT == 1) {
+    const int wi = idx >> 1;
+    const uint32_t wd = wi == 0 ? h.x : wi == 1 ? h.y : wi == 2 ? h.z : h.w;
+    return (idx & 1) ? bf16hi(wd) : bf16lo(wd);
+  } else {
+    return __uint_as_float(idx == 0 ? h.x : idx == 1 ? h.y : idx == 2 ? h.z : h.w);
+  }
+}
+
+// If this thread's group (units u, u + kThreads, ...) holds the drafted token,
+// take its logit from the registers.
+template <int DT, int N>
+__device__ __forceinline__ void pick_token(const uint4 (&v)[N], int u, int tok, float& xv, bool& hit) {
+  constexpr int E = Elem<DT>::kPerVec;
+  if (tok < 0) return;
+  const int rel = tok / E - u;
+  if (rel >= 0 && rel < N * kThreads && rel % kThreads == 0) {
+    uint4 h = v[0];
+#pragma unroll
+    for (int t = 1; t < N; ++t)
+      if (rel == t * kThreads) h = v[t];
+    xv = vec_elem<DT>(h, tok - (tok / E) * E);
+    hit = true;
+  }
+}
+
+// Vector path: each segment (the block's part of one row) streams groups of
+// kUnroll 16-byte vectors per thread, then single vectors, and ends with one
+// block merge. The drafted token is loaded with the row's first data and
+// used only after it, so the stream never waits on it.
+template <int DT>
+__device__ __forceinline__ void walk_vec(const RowSpace& rs, const Walk& w, int64_t Vu, int64_t e0, int64_t e1,
+                                         float k, float2* __restrict__ part, float2* red) {
+  const int tid = threadIdx.x;
+  for (int64_t e = e0; e < e1;) {
+    const int64_t r = e / Vu;
+    const int u0 = static_cast<int>(e - r * Vu), u1 = static_cast<int>(min(e1, (r + 1) * Vu) - r * Vu);
+    const int32_t* tokp;
+    const uint4* rv = reinterpret_cast<const uint4*>(locate<DT>(rs, w, r, tokp));
+    const int tok = load_token(tokp);  // out of range: matches no unit of the row
+    float m = -INFINITY, s = 0.f, xv = 0.f;
+    bool hit = false;
+    int u = u0 + tid;
     for (; u + (kUnroll - 1) * kThreads < u1; u += kUnroll * kThreads) {
       uint4 v[kUnroll];
 #pragma unroll
       for (int t = 0; t < kUnroll; ++t) v[t] = ldg16(rv + u + t * kThreads);
       fold_vectors<DT, kUnroll>(v, m, s, k);
+      pick_token<DT, kUnroll>(v, u, tok, xv, hit);
     }
     for (; u < u1; u += kThreads) {
-      uint4 v[1] = {ldg16(rv + u)};
+      const uint4 v[1] = {ldg16(rv + u)};
       fold_vectors<DT, 1>(v, m, s, k);
+      pick_token<DT, 1>(v, u, tok, xv, hit);
     }
-  } else {
-    for (; u < u1; u += kThreads) {
+    if (hit) rs.xg[r] = xv;
+    block_merge(m, s, k, red);
+    if (tid == 0) part[blockIdx.x + r] = make_float2(m, s);
+    e = r * Vu + u1;
+  }
+}
+
+// Scalar path (rows that are not 16-byte vectors): one segment at a time.
+template <int DT>
+__device__ __forceinline__ void walk_scalar(const RowSpace& rs, const Walk& w, int64_t Vu, int64_t e0, int64_t e1,
+                                            float k, float2* __restrict__ part, float2* red) {
+  for (int64_t e = e0; e < e1;) {
+    const int64_t r = e / Vu;
+    const int64_t se = min(e1, (r + 1) * Vu);
+    const int32_t* tokp;
+    const char* row = locate<DT>(rs, w, r, tokp);
+    const int tok = load_token(tokp);
+    float m = -INFINITY, s = 0.f;
+    for (int64_t u = e - r * Vu + threadIdx.x; u < se - r * Vu; u += kThreads) {
       const float x = Elem<DT>::at(row, u);
       if (x > m) {
         s *= ex2((m - x) * k);
         m = x;
       }
       if (m != -INFINITY) s += ex2((x - m) * k);
+      if (u == tok) rs.xg[r] = x;
     }
+    block_merge(m, s, k, red);
+    if (threadIdx.x == 0) part[blockIdx.x + r] = make_float2(m, s);
+    e = se;
   }
 }
 
 template <int DT, bool VEC>
 __global__ void __launch_bounds__(kThreads) k_row_stats(RowSpace rs, int64_t Vu, int G, float k,
                                                         float2* __restrict__ part) {
-  extern __shared__ int rowoff[];
+  extern __shared__ int walk_smem[];  // verify mode: rowoff[B + 1], base[B]
   __shared__ float2 red[kWarps];
   __shared__ int tmp[kWarps + 1];
   pdl_wait();
   pdl_trigger();
   int64_t nrows;
+  Walk w{walk_smem, walk_smem + rs.B + 1};
   if (rs.verify) {
+    int* rowoff = walk_smem;
+    int* base = walk_smem + rs.B + 1;
     for (int b = threadIdx.x; b < rs.B; b += kThreads) {
       int l = rs.vlen ? rs.vlen[b] : rs.L;
       if (l < 0 || l > rs.L) l = 0;  // flagged by the sampling kernel
       rowoff[b] = (rs.K + 1) * l;
+      base[b] = rs.row_off ? rs.row_off[b] : b * (rs.L + 1);
     }
     __syncthreads();
     nrows = block_exclusive_scan(rowoff, rs.B, tmp);
+    if (threadIdx.x == 0) rowoff[rs.B] = static_cast<int>(nrows);
+    __syncthreads();
   } else {
     nrows = rs.rows;
   }
   const int64_t N = nrows * Vu;
-  const int64_t e1 = split_start(blockIdx.x + 1, N, G);
-  for (int64_t e = split_start(blockIdx.x, N, G); e < e1;) {
-    const int64_t r = e / Vu;
-    const int64_t se = min(e1, (r + 1) * Vu);
-    int tok;
-    const char* row = row_pointer<DT>(rs, r, rowoff, tok);
-    float m = -INFINITY, s = 0.f;
-    segment_stats<DT, VEC>(row, e - r * Vu, se - r * Vu, k, m, s, tok, rs.xg ? rs.xg + r : nullptr);
-    block_merge(m, s, k, red);
-    if (threadIdx.x == 0) part[blockIdx.x + r] = make_float2(m, s);
-    e = se;
-  }
+  const int64_t e0 = split_start(blockIdx.x, N, G), e1 = split_start(blockIdx.x + 1, N, G);
+  if (e0 >= e1) return;  // empty share (N < grid): no partials
+  if constexpr (VEC) walk_vec<DT>(rs, w, Vu, e0, e1, k, part, red);
+  else walk_scalar<DT>(rs, w, Vu, e0, e1, k, part, red);
 }
 
 // Merge the partials of row r.
@@ -220,7 +285,7 @@ cudaError_t launch_row_stats(const RowSpace& rs, int dtype, bool vec, int64_t V,
                              cudaStream_t st) {
   const int64_t Vu = units_per_row(V, dtype, vec);
   const float k = log2e_over(T);
-  const size_t smem = rs.verify ? static_cast<size_t>(rs.B) * sizeof(int) : 0;
+  const size_t smem = rs.verify ? static_cast<size_t>(2 * rs.B + 1) * sizeof(int) : 0;
   const dim3 grid(G), block(kThreads);
   if (dtype == 0)
     return vec ? launch_pdl(k_row_stats<0, true>, grid, block, smem, st, rs, Vu, G, k, part)

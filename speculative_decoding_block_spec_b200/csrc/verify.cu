@@ -11,16 +11,19 @@
 //
 // Grid (P, B), launched after the statistics kernel with programmatic
 // dependent launch. The P blocks of request b each
+//   0. read the request's tokens, uniforms and mixture weights while the
+//      statistics kernel is still finishing;
 //   1. merge the statistics partials of the request's window rows and read the
 //      drafted-token logits the statistics kernel recorded;
-//   2. take the accept decisions in one warp (decide_warp) — identically in
-//      every block, so no block waits for another;
+//   2. take the accept decisions in one warp (decide_warp), identically in
+//      every block, so no block waits for another; block 0 then writes the
+//      accepted length and every output token but the terminal one;
 //   3. score 1/P of terminal row j (target, K draft rows, Gumbel row) and
 //      publish each warp's best residual and bonus candidates as 64-bit
 //      order-preserving keys with red.max (no return, no wait).
-// The last block of the grid to finish (atomic ticket) writes every
-// request's accepted length and tokens and clears the keys, so the workspace
-// is ready for the next call.
+// The last of the request's blocks to finish (per-request atomic ticket)
+// writes the terminal token and clears the request's keys and ticket, so the
+// workspace is ready for the next call.
 #include <algorithm>
 
 #include "common.cuh"
@@ -56,73 +59,86 @@ __device__ __forceinline__ int64_t owner_of(int64_t e, int64_t N, int64_t G) {
 }
 
 template <int DT, bool VEC>
-__global__ void __launch_bounds__(kThreads) k_accept_sample(VerifyArgs a, float k) {
+__global__ void __launch_bounds__(kThreads, 3) k_accept_sample(VerifyArgs a, float k) {
   __shared__ float s_xg[kMaxRows];  // logit at the drafted token, per request row
   __shared__ float s_m[kMaxRows], s_s[kMaxRows];
   __shared__ int s_x[kMaxL];
+  __shared__ float s_u[kMaxL], s_w[kMaxK];
   __shared__ float s_c[kMaxK + 1], s_mm[kMaxK + 1];
-  __shared__ int s_flags, s_j, s_last;
+  __shared__ int s_flags, s_j, s_last, s_fail;
   __shared__ int s_cnt[2 * kWarps];
 
   const int b = blockIdx.y, p = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
   const int L = a.L, K = a.K;
   const int64_t V = a.V;
+  int32_t* out = a.out_tokens + static_cast<int64_t>(b) * (L + 1);
 
+  // ---- 0. inputs that do not come from the statistics kernel: read while it
+  //         finishes (this grid starts early through programmatic launch)
   int ell = a.vlen ? a.vlen[b] : L;
   const bool bad_len = ell < 0 || ell > L;
   if (bad_len) ell = 0;
   if (tid == 0) s_flags = bad_len ? kFlagVerifyLen : 0;
   const int64_t toff = a.row_off ? static_cast<int64_t>(a.row_off[b]) : static_cast<int64_t>(b) * (L + 1);
-
-  pdl_wait();
-  pdl_trigger();
-
-  // ---- 1. this request's rows: offset in the statistics walk, partials, token logits
-  int before = 0, total = 0;
-  for (int bb = tid; bb < a.B; bb += kThreads) {
-    int l = a.vlen ? a.vlen[bb] : L;
-    if (l < 0 || l > L) l = 0;
-    total += l;
-    if (bb < b) before += l;
-  }
+  int before = b * L, total = a.B * L;  // verified positions of earlier requests, of all requests
+  if (a.vlen) {
+    before = 0;
+    total = 0;
+    for (int bb = tid; bb < a.B; bb += kThreads) {
+      int l = a.vlen[bb];
+      if (l < 0 || l > L) l = 0;
+      total += l;
+      if (bb < b) before += l;
+    }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    before += __shfl_xor_sync(0xffffffffu, before, o);
-    total += __shfl_xor_sync(0xffffffffu, total, o);
-  }
-  if (lane == 0) {
-    s_cnt[tid >> 5] = before;
-    s_cnt[kWarps + (tid >> 5)] = total;
+    for (int o = 16; o > 0; o >>= 1) {
+      before += __shfl_xor_sync(0xffffffffu, before, o);
+      total += __shfl_xor_sync(0xffffffffu, total, o);
+    }
+    if (lane == 0) {
+      s_cnt[tid >> 5] = before;
+      s_cnt[kWarps + (tid >> 5)] = total;
+    }
   }
   __syncthreads();
-  before = 0;
-  total = 0;
-  for (int w = 0; w < kWarps; ++w) {
-    before += s_cnt[w];
-    total += s_cnt[kWarps + w];
+  if (a.vlen) {
+    before = 0;
+    total = 0;
+    for (int w = 0; w < kWarps; ++w) {
+      before += s_cnt[w];
+      total += s_cnt[kWarps + w];
+    }
   }
-  const int nb = (K + 1) * ell;
-  const int64_t rowbase = static_cast<int64_t>(before) * (K + 1);
-  const int64_t N = static_cast<int64_t>(total) * (K + 1) * a.Vu;
   if (tid < ell) {
     const int x = a.tokens[static_cast<int64_t>(b) * L + tid];
     if (x < 0 || x >= V) atomicOr(&s_flags, kFlagTokenRange);
     s_x[tid] = x;
+    s_u[tid] = a.u[static_cast<int64_t>(b) * L + tid];
   }
+  if (tid < K && a.mix_w) s_w[tid] = a.mix_w[static_cast<int64_t>(b) * K + tid];
+
+  pdl_wait();
+  pdl_trigger();
+
+  // ---- 1. this request's rows: merge the statistics partials (one round trip
+  //         for up to 8 partials per row) and read the drafted-token logits
+  const int nb = (K + 1) * ell;
+  const int64_t rowbase = static_cast<int64_t>(before) * (K + 1);
+  const int64_t N = static_cast<int64_t>(total) * (K + 1) * a.Vu;
   for (int q = tid; q < nb; q += kThreads) {
     const int64_t r = rowbase + q;
     const int64_t c0 = owner_of(r * a.Vu, N, a.G), c1 = owner_of((r + 1) * a.Vu - 1, N, a.G);
     const float xq = __ldcg(a.xg + r);
     float m = -INFINITY, s = 0.f;
-    for (int64_t c = c0; c <= c1; c += 4) {  // 4 independent loads in flight per round trip
-      float2 pr[4];
+    for (int64_t c = c0; c <= c1; c += 8) {
+      float2 pr[8];
 #pragma unroll
-      for (int t = 0; t < 4; ++t)  // blocks with an empty share (only when N < grid) wrote nothing
+      for (int t = 0; t < 8; ++t)  // blocks with an empty share (only when N < grid) wrote nothing
         pr[t] = c + t <= c1 && (N >= a.G || split_start(c + t + 1, N, a.G) > split_start(c + t, N, a.G))
                     ? __ldcg(a.rpart + c + t + r)
                     : make_float2(-INFINITY, 0.f);
 #pragma unroll
-      for (int t = 0; t < 4; ++t) ms_merge(m, s, pr[t].x, pr[t].y, k);
+      for (int t = 0; t < 8; ++t) ms_merge(m, s, pr[t].x, pr[t].y, k);
     }
     s_m[q] = m;
     s_s[q] = s;
@@ -131,16 +147,16 @@ __global__ void __launch_bounds__(kThreads) k_accept_sample(VerifyArgs a, float 
   }
   __syncthreads();
 
-  // ---- 2. accept tests, first rejection by ballot
+  // ---- 2. accept tests and first rejection (warp 0, identically in every
+  //         block); block 0 then writes every output but the terminal token
   if (tid < 32) {
-    int j = ell;
-    if (s_flags == 0) {
+    int j = ell, f = s_flags;
+    if (f == 0) {
       const DecideIn in{s_xg, s_m, s_s, s_x, ell, K, L, a.T};
-      const DecideOut o = decide_warp(in, a.u + static_cast<int64_t>(b) * L,
-                                      a.mix_w ? a.mix_w + static_cast<int64_t>(b) * K : nullptr);
+      const DecideOut o = decide_warp(in, s_u, a.mix_w ? s_w : nullptr);
       j = o.j;
+      if (o.bad) f |= kFlagNonFinite;
       if (lane == 0) {
-        if (o.bad) s_flags |= kFlagNonFinite;
         s_c[0] = o.ct;
         s_mm[0] = o.mt;
         for (int z = 0; z < K; ++z) {
@@ -151,10 +167,16 @@ __global__ void __launch_bounds__(kThreads) k_accept_sample(VerifyArgs a, float 
     }
     if (lane == 0) {
       s_j = j;
-      if (p == 0) {  // for the block that writes the outputs
-        a.dec[b].j = j;
-        a.dec[b].flags = s_flags;
+      s_flags = f;
+    }
+    if (p == 0) {
+      for (int i = lane; i <= L; i += 32)
+        if (f || i != j) out[i] = (f == 0 && i < j) ? s_x[i] : -1;
+      if (lane == 0) {
+        a.accept_len[b] = f ? -1 : j;
+        if (f) atomicOr(a.status, f);
       }
+      __threadfence();  // ordered before this block's ticket
     }
   }
   __syncthreads();
@@ -218,35 +240,47 @@ __global__ void __launch_bounds__(kThreads) k_accept_sample(VerifyArgs a, float 
     if (lane == 0) {
       if (br.idx >= 0) red_max_u64(a.keys + 2 * b, score_key(br.score, br.idx));
       if (bb.idx >= 0) red_max_u64(a.keys + 2 * b + 1, score_key(bb.score, bb.idx));
+      __threadfence();  // the keys, before this block's ticket
     }
   }
 
-  // ---- the last block of the grid writes every request's outputs
-  __threadfence();
+  // ---- 4. the last of the request's P blocks writes its terminal token
   __syncthreads();
-  if (tid == 0) s_last = atomicAdd(a.tickets, 1) == static_cast<int>(gridDim.x * gridDim.y) - 1;
+  if (tid == 0) {
+    s_last = atomicAdd(a.tickets + b, 1) == a.P - 1;
+    s_fail = 0;
+  }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
-  for (int t = tid; t < a.B * (L + 1); t += kThreads) {
-    const int rb = t / (L + 1), i = t - rb * (L + 1);
-    int l = a.vlen ? a.vlen[rb] : L;
-    if (l < 0 || l > L) l = 0;
-    const int j = __ldcg(&a.dec[rb].j), f = __ldcg(&a.dec[rb].flags);
-    const unsigned long long kr = __ldcg(a.keys + 2 * rb), kb = __ldcg(a.keys + 2 * rb + 1);
-    const int tk = i < j ? __ldg(a.tokens + static_cast<int64_t>(rb) * L + i) : -1;
-    const int term = f ? -1 : ((j < l && kr) ? key_token(kr) : key_token(kb));
-    const bool ok = f == 0 && term >= 0;
-    a.out_tokens[static_cast<int64_t>(rb) * (L + 1) + i] = !ok ? -1 : (i < j ? tk : (i == j ? term : -1));
-    if (i == 0) {
-      a.accept_len[rb] = ok ? j : -1;
-      if (f) atomicOr(a.status, f);
-      else if (!ok) atomicOr(a.status, kFlagNonFinite);
+  if (tid == 0) {
+    __threadfence();
+    if (flags == 0) {
+      const int j = s_j;
+      const unsigned long long kr = __ldcg(a.keys + 2 * b), kb = __ldcg(a.keys + 2 * b + 1);
+      const int term = (j < ell && kr) ? key_token(kr) : key_token(kb);
+      if (term >= 0) out[j] = term;
+      else s_fail = 1;
+    }
+    a.keys[2 * b] = 0ull;
+    a.keys[2 * b + 1] = 0ull;
+    a.tickets[b] = 0;
+  }
+  __syncthreads();
+  if (s_fail) {  // no finite candidate in the terminal row: the request fails as a whole
+    for (int i = tid; i <= L; i += kThreads) out[i] = -1;
+    if (tid == 0) {
+      a.accept_len[b] = -1;
+      atomicOr(a.status, kFlagNonFinite);
     }
   }
-  __syncthreads();  // every output thread has read the keys before they are cleared
-  for (int t = tid; t < 2 * a.B; t += kThreads) a.keys[t] = 0ull;
-  if (tid == 0) *a.tickets = 0;
+}
+
+int accept_blocks_per_sm(int dtype, bool vec) {
+  int occ = 0;
+  cudaError_t e;
+  if (dtype == 0) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, vec ? k_accept_sample<0, true> : k_accept_sample<0, false>, kThreads, 0);
+  else e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, vec ? k_accept_sample<1, true> : k_accept_sample<1, false>, kThreads, 0);
+  return (e == cudaSuccess && occ > 0) ? occ : 1;
 }
 
 cudaError_t launch_accept_sample(const VerifyArgs& a, int dtype, bool vec, cudaStream_t st) {
