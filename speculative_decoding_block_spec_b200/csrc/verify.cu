@@ -32,6 +32,8 @@
 
 namespace specv {
 
+constexpr int kDraftBatch = 4;  // draft categories loaded together per terminal unit
+
 // Order-preserving 64-bit key of a terminal candidate: the fp64 score with its
 // lowest 20 bits replaced by (2^20 - 1 - token), so that an unsigned max picks
 // the highest score and, among scores equal to 32 significant bits, the lowest
@@ -194,19 +196,41 @@ __global__ void __launch_bounds__(kThreads, 3) k_accept_sample(VerifyArgs a, flo
     const int64_t Vu = V / E;
     const int64_t u1 = (static_cast<int64_t>(p) + 1) * Vu / a.P;
     Best br{-INFINITY, -1}, bb{-INFINITY, -1};
+    const char* dbase =
+        static_cast<const char*>(a.draft) + (static_cast<int64_t>(b) * K * L + j) * V * Elem<DT>::kBytes;
+    const int64_t dstride = static_cast<int64_t>(L) * V * Elem<DT>::kBytes;  // between draft categories
     for (int64_t u = static_cast<int64_t>(p) * Vu / a.P + tid; u < u1; u += kThreads) {
+      // every load of the unit is issued before any is used: one memory round
+      // trip per unit for up to kDraftBatch draft categories
       float xt[E], gv[E], q[E];
+      uint4 tv, gw[VEC ? E / 4 : 1], dv[kDraftBatch];
+      float xs = 0.f, gs = 0.f, ds[kDraftBatch];
       if constexpr (VEC) {
-        Elem<DT>::unpack(ldg16(reinterpret_cast<const uint4*>(trow) + u), xt);
+        tv = ldg16(reinterpret_cast<const uint4*>(trow) + u);
+#pragma unroll
+        for (int h = 0; h < E / 4; ++h) gw[h] = ldg16(reinterpret_cast<const uint4*>(grow + u * E) + h);
+      } else {
+        xs = Elem<DT>::at(trow, u);
+        gs = __ldg(grow + u);
+      }
+      if (resid) {
+#pragma unroll
+        for (int z = 0; z < kDraftBatch; ++z)
+          if (z < K) {
+            if constexpr (VEC) dv[z] = ldg16(reinterpret_cast<const uint4*>(dbase + z * dstride) + u);
+            else ds[z] = Elem<DT>::at(dbase + z * dstride, u);
+          }
+      }
+      if constexpr (VEC) {
+        Elem<DT>::unpack(tv, xt);
 #pragma unroll
         for (int h = 0; h < E / 4; ++h) {
-          const uint4 w = ldg16(reinterpret_cast<const uint4*>(grow + u * E) + h);
-          gv[4 * h] = __uint_as_float(w.x); gv[4 * h + 1] = __uint_as_float(w.y);
-          gv[4 * h + 2] = __uint_as_float(w.z); gv[4 * h + 3] = __uint_as_float(w.w);
+          gv[4 * h] = __uint_as_float(gw[h].x); gv[4 * h + 1] = __uint_as_float(gw[h].y);
+          gv[4 * h + 2] = __uint_as_float(gw[h].z); gv[4 * h + 3] = __uint_as_float(gw[h].w);
         }
       } else {
-        xt[0] = Elem<DT>::at(trow, u);
-        gv[0] = __ldg(grow + u);
+        xt[0] = xs;
+        gv[0] = gs;
       }
 #pragma unroll
       for (int e = 0; e < E; ++e) {
@@ -215,15 +239,33 @@ __global__ void __launch_bounds__(kThreads, 3) k_accept_sample(VerifyArgs a, flo
         q[e] = 0.f;
       }
       if (resid) {
-        for (int z = 0; z < K; ++z) {
-          const char* drow =
-              static_cast<const char*>(a.draft) + ((static_cast<int64_t>(b) * K + z) * L + j) * V * Elem<DT>::kBytes;
-          float xd[E];
-          if constexpr (VEC) Elem<DT>::unpack(ldg16(reinterpret_cast<const uint4*>(drow) + u), xd);
-          else xd[0] = Elem<DT>::at(drow, u);
-          const float cz = s_c[1 + z], mz = s_mm[1 + z];
 #pragma unroll
-          for (int e = 0; e < E; ++e) q[e] = fmaf(cz, ex2((xd[e] - mz) * k), q[e]);
+        for (int z = 0; z < kDraftBatch; ++z)
+          if (z < K) {
+            float xd[E];
+            if constexpr (VEC) Elem<DT>::unpack(dv[z], xd);
+            else xd[0] = ds[z];
+            const float cz = s_c[1 + z], mz = s_mm[1 + z];
+#pragma unroll
+            for (int e = 0; e < E; ++e) q[e] = fmaf(cz, ex2((xd[e] - mz) * k), q[e]);
+          }
+        for (int z0 = kDraftBatch; z0 < K; z0 += kDraftBatch) {  // K > kDraftBatch: further round trips
+#pragma unroll
+          for (int z = 0; z < kDraftBatch; ++z)
+            if (z0 + z < K) {
+              if constexpr (VEC) dv[z] = ldg16(reinterpret_cast<const uint4*>(dbase + (z0 + z) * dstride) + u);
+              else ds[z] = Elem<DT>::at(dbase + (z0 + z) * dstride, u);
+            }
+#pragma unroll
+          for (int z = 0; z < kDraftBatch; ++z)
+            if (z0 + z < K) {
+              float xd[E];
+              if constexpr (VEC) Elem<DT>::unpack(dv[z], xd);
+              else xd[0] = ds[z];
+              const float cz = s_c[1 + z0 + z], mz = s_mm[1 + z0 + z];
+#pragma unroll
+              for (int e = 0; e < E; ++e) q[e] = fmaf(cz, ex2((xd[e] - mz) * k), q[e]);
+            }
         }
 #pragma unroll
         for (int e = 0; e < E; ++e) {
