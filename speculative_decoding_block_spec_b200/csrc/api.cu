@@ -139,7 +139,8 @@ int launch_stats_stage(const void* target, const int32_t* row_off, const void* d
   rs.L = L;
   rs.K = K;
   rs.verify = 1;
-  const int G = stats_grid(dtype, vec, static_cast<int64_t>(B) * (K + 1) * L * units_per_row(V, dtype, vec));
+  const int64_t Vu = units_per_row(V, dtype, vec);
+  const int G = stats_grid(dtype, vec, static_cast<int64_t>(B) * (K + 1) * L * Vu, Vu);
   return map_cuda(launch_row_stats(rs, dtype, vec, V, T, G, reinterpret_cast<float2*>(static_cast<char*>(ws) + lay.rpart), st));
 }
 
@@ -173,7 +174,7 @@ int launch_accept_stage(const void* target, const int32_t* row_off, const void* 
   a.xg = reinterpret_cast<const float*>(w + lay.xg);
   a.rpart = reinterpret_cast<const float2*>(w + lay.rpart);
   a.Vu = units_per_row(V, dtype, vec);
-  a.G = stats_grid(dtype, vec, static_cast<int64_t>(B) * (K + 1) * L * a.Vu);
+  a.G = stats_grid(dtype, vec, static_cast<int64_t>(B) * (K + 1) * L * a.Vu, a.Vu);
   // Blocks per request for the terminal row: the whole (P, B) grid resident
   // at once (no second wave), at least 256 units of the row per block.
   const int64_t term_units = vec_term ? V / (16 / esize(dtype)) : V;
@@ -251,7 +252,7 @@ int spec_softmax_T(const void* logits, int dtype, int64_t rows, int64_t V, int64
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   float2* part = reinterpret_cast<float2*>(static_cast<char*>(workspace) + kHeader);
   const int64_t Vu = units_per_row(V, dtype, vec);
-  const int G = stats_grid(dtype, vec, rows * Vu);
+  const int G = stats_grid(dtype, vec, rows * Vu, Vu);
   RowSpace rs = {};
   rs.target = logits;
   rs.stride = row_stride;
@@ -281,7 +282,7 @@ int spec_softmax_T_noalloc(const void* logits, int dtype, int64_t rows, int64_t 
                    (!probs || aligned(probs, 16));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t Vu = units_per_row(V, dtype, vec);
-  const int G = stats_grid(dtype, vec, rows * Vu);
+  const int G = stats_grid(dtype, vec, rows * Vu, Vu);
   RowSpace rs = {};
   rs.target = logits;
   rs.stride = row_stride;

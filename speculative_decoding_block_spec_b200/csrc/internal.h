@@ -55,8 +55,8 @@ inline int64_t units_per_row(int64_t V, int dtype, bool vec) {
   return vec ? V * (dtype == 0 ? 4 : 2) / 16 : V;
 }
 
-// Grid size of the persistent row-statistics kernel for up to max_units units.
-int stats_grid(int dtype, bool vec, int64_t max_units);
+// Grid size of the row-statistics kernel for up to max_units units (Vu per row).
+int stats_grid(int dtype, bool vec, int64_t max_units, int64_t Vu);
 
 cudaError_t launch_row_stats(const RowSpace& rs, int dtype, bool vec, int64_t V, float T, int G,
                              float2* part, cudaStream_t st);

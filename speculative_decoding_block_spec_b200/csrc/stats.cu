@@ -60,67 +60,42 @@ __device__ __forceinline__ const char* locate(const RowSpace& rs, const Walk& w,
 
 __device__ __forceinline__ int load_token(const int32_t* tokp) { return tokp ? __ldg(tokp) : -1; }
 
-// Element `idx` (0..E-1) of a 16-byte vector.
-template <int DT>
-__device__ __forceinline__ float vec_elem(const uint4& h, int idx) {
-  if constexpr (DT == 1) {
-    const int wi = idx >> 1;
-    const uint32_t wd = wi == 0 ? h.x : wi == 1 ? h.y : wi == 2 ? h.z : h.w;
-    return (idx & 1) ? bf16hi(wd) : bf16lo(wd);
-  } else {
-    return __uint_as_float(idx == 0 ? h.x : idx == 1 ? h.y : idx == 2 ? h.z : h.w);
-  }
-}
-
-// If this thread's group (units u, u + kThreads, ...) holds the drafted token,
-// take its logit from the registers.
-template <int DT, int N>
-__device__ __forceinline__ void pick_token(const uint4 (&v)[N], int u, int tok, float& xv, bool& hit) {
-  constexpr int E = Elem<DT>::kPerVec;
-  if (tok < 0) return;
-  const int rel = tok / E - u;
-  if (rel >= 0 && rel < N * kThreads && rel % kThreads == 0) {
-    uint4 h = v[0];
-#pragma unroll
-    for (int t = 1; t < N; ++t)
-      if (rel == t * kThreads) h = v[t];
-    xv = vec_elem<DT>(h, tok - (tok / E) * E);
-    hit = true;
-  }
-}
-
 // Vector path: each segment (the block's part of one row) streams groups of
 // kUnroll 16-byte vectors per thread, then single vectors, and ends with one
-// block merge. The drafted token is loaded with the row's first data and
-// used only after it, so the stream never waits on it.
+// block merge. The drafted token is loaded with the row's first data; after
+// the segment, the thread whose units hold it re-reads that element (the row
+// has just passed through L2) and stores it once the merge is done, so
+// neither load stalls the stream.
 template <int DT>
 __device__ __forceinline__ void walk_vec(const RowSpace& rs, const Walk& w, int64_t Vu, int64_t e0, int64_t e1,
                                          float k, float2* __restrict__ part, float2* red) {
+  constexpr int E = Elem<DT>::kPerVec;
   const int tid = threadIdx.x;
   for (int64_t e = e0; e < e1;) {
     const int64_t r = e / Vu;
     const int u0 = static_cast<int>(e - r * Vu), u1 = static_cast<int>(min(e1, (r + 1) * Vu) - r * Vu);
     const int32_t* tokp;
-    const uint4* rv = reinterpret_cast<const uint4*>(locate<DT>(rs, w, r, tokp));
-    const int tok = load_token(tokp);  // out of range: matches no unit of the row
-    float m = -INFINITY, s = 0.f, xv = 0.f;
-    bool hit = false;
+    const char* row = locate<DT>(rs, w, r, tokp);
+    const uint4* rv = reinterpret_cast<const uint4*>(row);
+    const int tok = load_token(tokp);
+    float m = -INFINITY, s = 0.f;
     int u = u0 + tid;
     for (; u + (kUnroll - 1) * kThreads < u1; u += kUnroll * kThreads) {
       uint4 v[kUnroll];
 #pragma unroll
       for (int t = 0; t < kUnroll; ++t) v[t] = ldg16(rv + u + t * kThreads);
       fold_vectors<DT, kUnroll>(v, m, s, k);
-      pick_token<DT, kUnroll>(v, u, tok, xv, hit);
     }
     for (; u < u1; u += kThreads) {
       const uint4 v[1] = {ldg16(rv + u)};
       fold_vectors<DT, 1>(v, m, s, k);
-      pick_token<DT, 1>(v, u, tok, xv, hit);
     }
-    if (hit) rs.xg[r] = xv;
+    const int tu = tok / E;  // tok < 0: no token; tok >= V: matches no unit
+    const bool hit = tok >= 0 && tu >= u0 && tu < u1 && (tu - u0) % kThreads == tid;
+    const float xv = hit ? Elem<DT>::at(row, tok) : 0.f;
     block_merge(m, s, k, red);
     if (tid == 0) part[blockIdx.x + r] = make_float2(m, s);
+    if (hit) rs.xg[r] = xv;
     e = r * Vu + u1;
   }
 }
@@ -151,6 +126,26 @@ __device__ __forceinline__ void walk_scalar(const RowSpace& rs, const Walk& w, i
   }
 }
 
+// Rows of the walk; in verify mode also builds its geometry in shared memory
+// (every thread of the block calls this).
+template <int NT>
+__device__ __forceinline__ int64_t build_walk(const RowSpace& rs, int* walk_smem, int* tmp) {
+  if (!rs.verify) return rs.rows;
+  int* rowoff = walk_smem;
+  int* base = walk_smem + rs.B + 1;
+  for (int b = threadIdx.x; b < rs.B; b += NT) {
+    int l = rs.vlen ? rs.vlen[b] : rs.L;
+    if (l < 0 || l > rs.L) l = 0;  // flagged by the sampling kernel
+    rowoff[b] = (rs.K + 1) * l;
+    base[b] = rs.row_off ? rs.row_off[b] : b * (rs.L + 1);
+  }
+  __syncthreads();
+  const int64_t nrows = block_exclusive_scan<NT>(rowoff, rs.B, tmp);
+  if (threadIdx.x == 0) rowoff[rs.B] = static_cast<int>(nrows);
+  __syncthreads();
+  return nrows;
+}
+
 template <int DT, bool VEC>
 __global__ void __launch_bounds__(kThreads) k_row_stats(RowSpace rs, int64_t Vu, int G, float k,
                                                         float2* __restrict__ part) {
@@ -159,29 +154,155 @@ __global__ void __launch_bounds__(kThreads) k_row_stats(RowSpace rs, int64_t Vu,
   __shared__ int tmp[kWarps + 1];
   pdl_wait();
   pdl_trigger();
-  int64_t nrows;
-  Walk w{walk_smem, walk_smem + rs.B + 1};
-  if (rs.verify) {
-    int* rowoff = walk_smem;
-    int* base = walk_smem + rs.B + 1;
-    for (int b = threadIdx.x; b < rs.B; b += kThreads) {
-      int l = rs.vlen ? rs.vlen[b] : rs.L;
-      if (l < 0 || l > rs.L) l = 0;  // flagged by the sampling kernel
-      rowoff[b] = (rs.K + 1) * l;
-      base[b] = rs.row_off ? rs.row_off[b] : b * (rs.L + 1);
-    }
-    __syncthreads();
-    nrows = block_exclusive_scan(rowoff, rs.B, tmp);
-    if (threadIdx.x == 0) rowoff[rs.B] = static_cast<int>(nrows);
-    __syncthreads();
-  } else {
-    nrows = rs.rows;
-  }
-  const int64_t N = nrows * Vu;
+  const Walk w{walk_smem, walk_smem + rs.B + 1};
+  const int64_t N = build_walk<kThreads>(rs, walk_smem, tmp) * Vu;
   const int64_t e0 = split_start(blockIdx.x, N, G), e1 = split_start(blockIdx.x + 1, N, G);
   if (e0 >= e1) return;  // empty share (N < grid): no partials
   if constexpr (VEC) walk_vec<DT>(rs, w, Vu, e0, e1, k, part, red);
   else walk_scalar<DT>(rs, w, Vu, e0, e1, k, part, red);
+}
+
+// ------------------------------------------------ balanced vector kernel
+//
+// One block of kDynThreads per SM, each block with an even share of the
+// flattened units as above. Inside the block the share is cut into slices of
+// kSlice units that never cross a row (a row's piece of the share is a
+// segment); warps take slices in order from a shared-memory counter, with
+// the next slice's loads in flight while the current one is folded, so every
+// warp of an SM streams until the share is exhausted and the block ends
+// within about one slice of its fastest warp. A warp folds the slices of one
+// segment into its own (max, sum); when it moves on it stores that pair in
+// a [warp][segment] table, and the block merges each segment's column into
+// the (block, row) partial at the end. Used when a share spans at most
+// kMaxSegs rows.
+constexpr int kDynThreads = 1024;
+constexpr int kDynWarps = kDynThreads / 32;
+constexpr int kMaxSegs = 32;
+constexpr int kSliceVec = 4;              // 16-byte vectors per lane per slice
+constexpr int kSlice = 32 * kSliceVec;    // units per slice
+
+__device__ __forceinline__ void warp_merge(float& m, float& s, float k) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    ms_merge(m, s, m2, s2, k);
+  }
+}
+
+// Lane's vectors of slice position g (row-relative unit of lane 0), -inf past `end`.
+template <int DT>
+__device__ __forceinline__ void load_slice(const char* row, int g, int end, uint4 (&v)[kSliceVec]) {
+  const uint4* rv = reinterpret_cast<const uint4*>(row);
+  const uint32_t ninf = DT == 1 ? 0xFF80FF80u : 0xFF800000u;  // four or eight -inf: add nothing
+#pragma unroll
+  for (int t = 0; t < kSliceVec; ++t) {
+    const int u = g + t * 32;
+    v[t] = u < end ? ldg16(rv + u) : make_uint4(ninf, ninf, ninf, ninf);
+  }
+}
+
+template <int DT>
+__global__ void __launch_bounds__(kDynThreads, 1) k_row_stats_dyn(RowSpace rs, int64_t Vu, int G, float k,
+                                                                  float2* __restrict__ part) {
+  constexpr int E = Elem<DT>::kPerVec;
+  extern __shared__ int walk_smem[];  // verify mode: rowoff[B + 1], base[B]
+  __shared__ float2 s_tab[kDynWarps][kMaxSegs];
+  __shared__ const char* s_ptr[kMaxSegs];
+  __shared__ const int32_t* s_tokp[kMaxSegs];
+  __shared__ int s_a[kMaxSegs], s_b[kMaxSegs], s_first[kMaxSegs + 1];
+  __shared__ int s_next;
+  __shared__ int tmp[kDynWarps + 1];
+  pdl_wait();
+  pdl_trigger();
+  const Walk w{walk_smem, walk_smem + rs.B + 1};
+  const int64_t N = build_walk<kDynThreads>(rs, walk_smem, tmp) * Vu;
+  const int64_t e0 = split_start(blockIdx.x, N, G), e1 = split_start(blockIdx.x + 1, N, G);
+  if (e0 >= e1) return;  // empty share (N < grid): no partials
+  const int64_t r0 = e0 / Vu;
+  const int nseg = static_cast<int>((e1 - 1) / Vu - r0 + 1);
+  if (nseg > kMaxSegs) return;  // excluded by the host's choice of kernel
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  if (tid < nseg) {
+    const int64_t r = r0 + tid;
+    s_a[tid] = static_cast<int>(max(e0, r * Vu) - r * Vu);
+    s_b[tid] = static_cast<int>(min(e1, (r + 1) * Vu) - r * Vu);
+    const int32_t* tp;
+    s_ptr[tid] = locate<DT>(rs, w, r, tp);
+    s_tokp[tid] = tp;
+  }
+  for (int i = tid; i < kDynWarps * kMaxSegs; i += kDynThreads) (&s_tab[0][0])[i] = make_float2(-INFINITY, 0.f);
+  if (tid == 0) s_next = 0;
+  __syncthreads();
+  if (tid < 32) {  // first slice of each segment (inclusive scan of slice counts)
+    int n = lane < nseg ? (s_b[lane] - s_a[lane] + kSlice - 1) / kSlice : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, n, o);
+      if (lane >= o) n += t;
+    }
+    s_first[lane + 1] = n;
+    if (lane == 0) s_first[0] = 0;
+  }
+  __syncthreads();
+  const int nslices = s_first[nseg];
+
+  // The last warp first records the drafted-token logit of every segment whose
+  // token falls in this block's share (two dependent loads), then joins the
+  // stream late; the other warps take the slices it does not.
+  if (wid == kDynWarps - 1 && lane < nseg) {
+    const int tok = load_token(s_tokp[lane]);
+    if (tok >= 0 && tok / E >= s_a[lane] && tok / E < s_b[lane]) rs.xg[r0 + lane] = Elem<DT>::at(s_ptr[lane], tok);
+  }
+
+  int seg = 0;  // this warp's segment cursor (slices are taken in increasing order)
+  int kc;
+  if (lane == 0) kc = atomicAdd(&s_next, 1);
+  kc = __shfl_sync(0xffffffffu, kc, 0);
+  uint4 vc[kSliceVec];
+  int segc = 0, gc = 0;
+  if (kc < nslices) {
+    while (s_first[seg + 1] <= kc) ++seg;
+    segc = seg;
+    gc = s_a[seg] + (kc - s_first[seg]) * kSlice + lane;
+    load_slice<DT>(s_ptr[seg], gc, s_b[seg], vc);
+  }
+  float m = -INFINITY, s = 0.f;
+  int acc = segc;
+  while (kc < nslices) {
+    int kn;
+    if (lane == 0) kn = atomicAdd(&s_next, 1);
+    kn = __shfl_sync(0xffffffffu, kn, 0);
+    uint4 vn[kSliceVec];
+    int segn = segc, gn = 0;
+    if (kn < nslices) {  // the next slice's loads go out before this one is folded
+      while (s_first[seg + 1] <= kn) ++seg;
+      segn = seg;
+      gn = s_a[seg] + (kn - s_first[seg]) * kSlice + lane;
+      load_slice<DT>(s_ptr[seg], gn, s_b[seg], vn);
+    }
+    if (segc != acc) {  // this warp is done with segment acc
+      warp_merge(m, s, k);
+      if (lane == 0) s_tab[wid][acc] = make_float2(m, s);
+      m = -INFINITY;
+      s = 0.f;
+      acc = segc;
+    }
+    fold_vectors<DT, kSliceVec>(vc, m, s, k);
+#pragma unroll
+    for (int t = 0; t < kSliceVec; ++t) vc[t] = vn[t];
+    kc = kn;
+    segc = segn;
+    gc = gn;
+  }
+  warp_merge(m, s, k);
+  if (lane == 0) s_tab[wid][acc] = make_float2(m, s);  // (-inf, 0) if this warp had no slice
+  __syncthreads();
+  for (int sg = wid; sg < nseg; sg += kDynWarps) {
+    float2 v = s_tab[lane][sg];
+    warp_merge(v.x, v.y, k);
+    if (lane == 0) part[blockIdx.x + r0 + sg] = v;
+  }
 }
 
 // Merge the partials of row r.
@@ -273,7 +394,34 @@ static int occupancy_of() {
   return g;
 }
 
-int stats_grid(int dtype, bool vec, int64_t max_units) {
+static int device_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  static std::mutex mu;
+  static int cache[64] = {0};
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 64 && cache[dev]) return cache[dev];
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) sms = 148;
+  if (dev < 64) cache[dev] = sms;
+  return sms;
+}
+
+// The balanced kernel runs one block per SM; it needs 16-byte vectors, a
+// share of at most kMaxSegs rows per block and at least one slice per warp.
+// It is chosen for windows of at most kDynMaxBytes: there the tail of
+// unevenly progressing blocks is a large part of the launch, and on B200 it
+// measured faster than the even split (78 MB: 21.5 against 23.0 us; 146 MB:
+// equal), while on windows of 0.7-0.8 GB the even split was as fast or faster.
+constexpr int64_t kDynMaxBytes = int64_t{256} << 20;
+
+static bool use_dyn(bool vec, int64_t max_units, int64_t Vu, int G) {
+  if (!vec || G != device_sms() || max_units * 16 > kDynMaxBytes) return false;
+  const int64_t share = (max_units + G - 1) / G;
+  return share >= static_cast<int64_t>(kDynThreads / 32) * kSlice && (share + Vu - 1) / Vu + 1 <= kMaxSegs;
+}
+
+int stats_grid(int dtype, bool vec, int64_t max_units, int64_t Vu) {
+  if (use_dyn(vec, max_units, Vu, device_sms())) return device_sms();
   int g;
   if (dtype == 0) g = vec ? occupancy_of<0, true>() : occupancy_of<0, false>();
   else g = vec ? occupancy_of<1, true>() : occupancy_of<1, false>();
@@ -287,6 +435,10 @@ cudaError_t launch_row_stats(const RowSpace& rs, int dtype, bool vec, int64_t V,
   const float k = log2e_over(T);
   const size_t smem = rs.verify ? static_cast<size_t>(2 * rs.B + 1) * sizeof(int) : 0;
   const dim3 grid(G), block(kThreads);
+  const int64_t max_units = (rs.verify ? static_cast<int64_t>(rs.B) * (rs.K + 1) * rs.L : rs.rows) * Vu;
+  if (use_dyn(vec, max_units, Vu, G))
+    return dtype == 0 ? launch_pdl(k_row_stats_dyn<0>, grid, dim3(kDynThreads), smem, st, rs, Vu, G, k, part)
+                      : launch_pdl(k_row_stats_dyn<1>, grid, dim3(kDynThreads), smem, st, rs, Vu, G, k, part);
   if (dtype == 0)
     return vec ? launch_pdl(k_row_stats<0, true>, grid, block, smem, st, rs, Vu, G, k, part)
                : launch_pdl(k_row_stats<0, false>, grid, block, smem, st, rs, Vu, G, k, part);
