@@ -51,6 +51,12 @@ __device__ __forceinline__ void red_max_u64(unsigned long long* p, unsigned long
   asm volatile("red.relaxed.gpu.global.max.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
+__device__ __forceinline__ int ticket_acq_rel(int* p) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+  return old;
+}
+
 // Owner block of unit e in the even split, without a 64-bit integer division.
 __device__ __forceinline__ int64_t owner_of(int64_t e, int64_t N, int64_t G) {
   const int64_t num = (e + 1) * G - 1;
@@ -178,7 +184,6 @@ __global__ void __launch_bounds__(kThreads, 3) k_accept_sample(VerifyArgs a, flo
         a.accept_len[b] = f ? -1 : j;
         if (f) atomicOr(a.status, f);
       }
-      __threadfence();  // ordered before this block's ticket
     }
   }
   __syncthreads();
@@ -282,20 +287,21 @@ __global__ void __launch_bounds__(kThreads, 3) k_accept_sample(VerifyArgs a, flo
     if (lane == 0) {
       if (br.idx >= 0) red_max_u64(a.keys + 2 * b, score_key(br.score, br.idx));
       if (bb.idx >= 0) red_max_u64(a.keys + 2 * b + 1, score_key(bb.score, bb.idx));
-      __threadfence();  // the keys, before this block's ticket
     }
   }
 
-  // ---- 4. the last of the request's P blocks writes its terminal token
+  // ---- 4. the last of the request's P blocks writes its terminal token. The
+  //         block barrier orders every thread's outputs and keys before thread
+  //         0's ticket, whose gpu-scope release publishes them and whose
+  //         acquire (in the last block) makes the other blocks' keys visible.
   __syncthreads();
   if (tid == 0) {
-    s_last = atomicAdd(a.tickets + b, 1) == a.P - 1;
+    s_last = ticket_acq_rel(a.tickets + b) == a.P - 1;
     s_fail = 0;
   }
   __syncthreads();
   if (!s_last) return;
   if (tid == 0) {
-    __threadfence();
     if (flags == 0) {
       const int j = s_j;
       const unsigned long long kr = __ldcg(a.keys + 2 * b), kb = __ldcg(a.keys + 2 * b + 1);
