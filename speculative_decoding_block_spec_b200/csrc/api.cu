@@ -57,15 +57,15 @@ int noalloc_scratch(float2** out) {
   return SPEC_OK;
 }
 
-// Resident sampling blocks per SM (cached per device and variant).
-int accept_slots(int dtype, bool vec) {
+// Resident sampling blocks per SM (cached per device and kernel variant).
+int accept_slots(int dtype, bool vec, int K) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
   static std::mutex mu;
-  static int cache[64][4] = {};
+  static int cache[64][8] = {};
   std::lock_guard<std::mutex> lock(mu);
-  int& c = cache[dev][dtype * 2 + (vec ? 1 : 0)];
-  if (!c) c = accept_blocks_per_sm(dtype, vec);
+  int& c = cache[dev][dtype * 4 + (vec ? 2 : 0) + (K == 1 ? 1 : 0)];
+  if (!c) c = accept_blocks_per_sm(dtype, vec, K);
   return c;
 }
 
@@ -178,7 +178,7 @@ int launch_accept_stage(const void* target, const int32_t* row_off, const void* 
   // Blocks per request for the terminal row: the whole (P, B) grid resident
   // at once (no second wave), at least 256 units of the row per block.
   const int64_t term_units = vec_term ? V / (16 / esize(dtype)) : V;
-  const int64_t slots = static_cast<int64_t>(sm_count()) * accept_slots(dtype, vec_term);
+  const int64_t slots = static_cast<int64_t>(sm_count()) * accept_slots(dtype, vec_term, K);
   const int64_t p_fit = std::max<int64_t>(1, slots / B);
   a.P = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({p_fit, kPMax, term_units / kThreads})));
   return map_cuda(launch_accept_sample(a, dtype, vec_term, st));

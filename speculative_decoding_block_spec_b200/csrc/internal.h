@@ -66,7 +66,7 @@ cudaError_t launch_softmax_finalize(const void* logits, int dtype, bool vec, int
                                     float* row_lse, float* probs, cudaStream_t st);
 
 cudaError_t launch_accept_sample(const VerifyArgs& a, int dtype, bool vec, cudaStream_t st);
-int accept_blocks_per_sm(int dtype, bool vec);
+int accept_blocks_per_sm(int dtype, bool vec, int K);
 
 cudaError_t launch_dvl(const float* scores, int B, int L, int budget, int32_t* verify_len,
                        int32_t* offsets, int32_t* slot_map, int* status, int* ticket,

@@ -32,8 +32,6 @@
 
 namespace specv {
 
-constexpr int kDraftBatch = 4;  // draft categories loaded together per terminal unit
-
 // Order-preserving 64-bit key of a terminal candidate: the fp64 score with its
 // lowest 20 bits replaced by (2^20 - 1 - token), so that an unsigned max picks
 // the highest score and, among scores equal to 32 significant bits, the lowest
@@ -66,7 +64,9 @@ __device__ __forceinline__ int64_t owner_of(int64_t e, int64_t N, int64_t G) {
   return q;
 }
 
-template <int DT, bool VEC>
+// KB: draft categories loaded together per terminal unit (1 for independent
+// drafts, which then take two units per thread per iteration; 4 otherwise).
+template <int DT, bool VEC, int KB>
 __global__ void __launch_bounds__(kThreads, 3) k_accept_sample(VerifyArgs a, float k) {
   __shared__ float s_xg[kMaxRows];  // logit at the drafted token, per request row
   __shared__ float s_m[kMaxRows], s_s[kMaxRows];
@@ -204,80 +204,92 @@ __global__ void __launch_bounds__(kThreads, 3) k_accept_sample(VerifyArgs a, flo
     const char* dbase =
         static_cast<const char*>(a.draft) + (static_cast<int64_t>(b) * K * L + j) * V * Elem<DT>::kBytes;
     const int64_t dstride = static_cast<int64_t>(L) * V * Elem<DT>::kBytes;  // between draft categories
-    for (int64_t u = static_cast<int64_t>(p) * Vu / a.P + tid; u < u1; u += kThreads) {
-      // every load of the unit is issued before any is used: one memory round
-      // trip per unit for up to kDraftBatch draft categories
-      float xt[E], gv[E], q[E];
-      uint4 tv, gw[VEC ? E / 4 : 1], dv[kDraftBatch];
-      float xs = 0.f, gs = 0.f, ds[kDraftBatch];
-      if constexpr (VEC) {
-        tv = ldg16(reinterpret_cast<const uint4*>(trow) + u);
+    // Every load of the kU units a thread takes per iteration is issued before
+    // any is used: one memory round trip per iteration for up to KB draft
+    // categories (further categories in batches of KB).
+    constexpr int kU = KB == 1 ? 2 : 1;
+    for (int64_t u0 = static_cast<int64_t>(p) * Vu / a.P + tid; u0 < u1; u0 += kU * kThreads) {
+      uint4 tv[kU], gw[kU][VEC ? E / 4 : 1], dv[kU][KB];
+      float xs[kU], gs[kU], ds[kU][KB];
 #pragma unroll
-        for (int h = 0; h < E / 4; ++h) gw[h] = ldg16(reinterpret_cast<const uint4*>(grow + u * E) + h);
-      } else {
-        xs = Elem<DT>::at(trow, u);
-        gs = __ldg(grow + u);
-      }
-      if (resid) {
+      for (int h = 0; h < kU; ++h) {
+        const int64_t u = u0 + h * kThreads;
+        if (u >= u1) break;
+        if constexpr (VEC) {
+          tv[h] = ldg16(reinterpret_cast<const uint4*>(trow) + u);
 #pragma unroll
-        for (int z = 0; z < kDraftBatch; ++z)
-          if (z < K) {
-            if constexpr (VEC) dv[z] = ldg16(reinterpret_cast<const uint4*>(dbase + z * dstride) + u);
-            else ds[z] = Elem<DT>::at(dbase + z * dstride, u);
-          }
-      }
-      if constexpr (VEC) {
-        Elem<DT>::unpack(tv, xt);
-#pragma unroll
-        for (int h = 0; h < E / 4; ++h) {
-          gv[4 * h] = __uint_as_float(gw[h].x); gv[4 * h + 1] = __uint_as_float(gw[h].y);
-          gv[4 * h + 2] = __uint_as_float(gw[h].z); gv[4 * h + 3] = __uint_as_float(gw[h].w);
+          for (int c = 0; c < E / 4; ++c) gw[h][c] = ldg16(reinterpret_cast<const uint4*>(grow + u * E) + c);
+        } else {
+          xs[h] = Elem<DT>::at(trow, u);
+          gs[h] = __ldg(grow + u);
         }
-      } else {
-        xt[0] = xs;
-        gv[0] = gs;
+        if (resid) {
+#pragma unroll
+          for (int z = 0; z < KB; ++z)
+            if (z < K) {
+              if constexpr (VEC) dv[h][z] = ldg16(reinterpret_cast<const uint4*>(dbase + z * dstride) + u);
+              else ds[h][z] = Elem<DT>::at(dbase + z * dstride, u);
+            }
+        }
       }
 #pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const Best c{static_cast<double>(xt[e]) * invT + static_cast<double>(gv[e]), static_cast<int>(u * E + e)};
-        if (c.score > bb.score) bb = c;
-        q[e] = 0.f;
-      }
-      if (resid) {
+      for (int h = 0; h < kU; ++h) {
+        const int64_t u = u0 + h * kThreads;
+        if (u >= u1) break;
+        float xt[E], gv[E], q[E];
+        if constexpr (VEC) {
+          Elem<DT>::unpack(tv[h], xt);
 #pragma unroll
-        for (int z = 0; z < kDraftBatch; ++z)
-          if (z < K) {
-            float xd[E];
-            if constexpr (VEC) Elem<DT>::unpack(dv[z], xd);
-            else xd[0] = ds[z];
-            const float cz = s_c[1 + z], mz = s_mm[1 + z];
-#pragma unroll
-            for (int e = 0; e < E; ++e) q[e] = fmaf(cz, ex2((xd[e] - mz) * k), q[e]);
+          for (int c = 0; c < E / 4; ++c) {
+            gv[4 * c] = __uint_as_float(gw[h][c].x); gv[4 * c + 1] = __uint_as_float(gw[h][c].y);
+            gv[4 * c + 2] = __uint_as_float(gw[h][c].z); gv[4 * c + 3] = __uint_as_float(gw[h][c].w);
           }
-        for (int z0 = kDraftBatch; z0 < K; z0 += kDraftBatch) {  // K > kDraftBatch: further round trips
-#pragma unroll
-          for (int z = 0; z < kDraftBatch; ++z)
-            if (z0 + z < K) {
-              if constexpr (VEC) dv[z] = ldg16(reinterpret_cast<const uint4*>(dbase + (z0 + z) * dstride) + u);
-              else ds[z] = Elem<DT>::at(dbase + (z0 + z) * dstride, u);
-            }
-#pragma unroll
-          for (int z = 0; z < kDraftBatch; ++z)
-            if (z0 + z < K) {
-              float xd[E];
-              if constexpr (VEC) Elem<DT>::unpack(dv[z], xd);
-              else xd[0] = ds[z];
-              const float cz = s_c[1 + z0 + z], mz = s_mm[1 + z0 + z];
-#pragma unroll
-              for (int e = 0; e < E; ++e) q[e] = fmaf(cz, ex2((xd[e] - mz) * k), q[e]);
-            }
+        } else {
+          xt[0] = xs[h];
+          gv[0] = gs[h];
         }
 #pragma unroll
         for (int e = 0; e < E; ++e) {
-          const float r = ex2((xt[e] - mt) * k) * ct - q[e];
-          if (r > 0.f) {
-            const Best c{static_cast<double>(lg2(r) * kLn2) + static_cast<double>(gv[e]), static_cast<int>(u * E + e)};
-            if (c.score > br.score) br = c;
+          const Best c{static_cast<double>(xt[e]) * invT + static_cast<double>(gv[e]), static_cast<int>(u * E + e)};
+          if (c.score > bb.score) bb = c;
+          q[e] = 0.f;
+        }
+        if (resid) {
+#pragma unroll
+          for (int z = 0; z < KB; ++z)
+            if (z < K) {
+              float xd[E];
+              if constexpr (VEC) Elem<DT>::unpack(dv[h][z], xd);
+              else xd[0] = ds[h][z];
+              const float cz = s_c[1 + z], mz = s_mm[1 + z];
+#pragma unroll
+              for (int e = 0; e < E; ++e) q[e] = fmaf(cz, ex2((xd[e] - mz) * k), q[e]);
+            }
+          for (int z0 = KB; z0 < K; z0 += KB) {  // K > KB: further round trips
+#pragma unroll
+            for (int z = 0; z < KB; ++z)
+              if (z0 + z < K) {
+                if constexpr (VEC) dv[h][z] = ldg16(reinterpret_cast<const uint4*>(dbase + (z0 + z) * dstride) + u);
+                else ds[h][z] = Elem<DT>::at(dbase + (z0 + z) * dstride, u);
+              }
+#pragma unroll
+            for (int z = 0; z < KB; ++z)
+              if (z0 + z < K) {
+                float xd[E];
+                if constexpr (VEC) Elem<DT>::unpack(dv[h][z], xd);
+                else xd[0] = ds[h][z];
+                const float cz = s_c[1 + z0 + z], mz = s_mm[1 + z0 + z];
+#pragma unroll
+                for (int e = 0; e < E; ++e) q[e] = fmaf(cz, ex2((xd[e] - mz) * k), q[e]);
+              }
+          }
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            const float r = ex2((xt[e] - mt) * k) * ct - q[e];
+            if (r > 0.f) {
+              const Best c{static_cast<double>(lg2(r) * kLn2) + static_cast<double>(gv[e]), static_cast<int>(u * E + e)};
+              if (c.score > br.score) br = c;
+            }
           }
         }
       }
@@ -323,22 +335,25 @@ __global__ void __launch_bounds__(kThreads, 3) k_accept_sample(VerifyArgs a, flo
   }
 }
 
-int accept_blocks_per_sm(int dtype, bool vec) {
+template <int DT, bool VEC>
+static auto accept_kernel(int K) {
+  return K == 1 ? k_accept_sample<DT, VEC, 1> : k_accept_sample<DT, VEC, 4>;
+}
+
+static auto accept_kernel(int dtype, bool vec, int K) {
+  if (dtype == 0) return vec ? accept_kernel<0, true>(K) : accept_kernel<0, false>(K);
+  return vec ? accept_kernel<1, true>(K) : accept_kernel<1, false>(K);
+}
+
+int accept_blocks_per_sm(int dtype, bool vec, int K) {
   int occ = 0;
-  cudaError_t e;
-  if (dtype == 0) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, vec ? k_accept_sample<0, true> : k_accept_sample<0, false>, kThreads, 0);
-  else e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, vec ? k_accept_sample<1, true> : k_accept_sample<1, false>, kThreads, 0);
+  const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, accept_kernel(dtype, vec, K), kThreads, 0);
   return (e == cudaSuccess && occ > 0) ? occ : 1;
 }
 
 cudaError_t launch_accept_sample(const VerifyArgs& a, int dtype, bool vec, cudaStream_t st) {
   const float k = static_cast<float>(1.4426950408889634 / static_cast<double>(a.T));
-  const dim3 grid(a.P, a.B), block(kThreads);
-  if (dtype == 0)
-    return vec ? launch_pdl(k_accept_sample<0, true>, grid, block, 0, st, a, k)
-               : launch_pdl(k_accept_sample<0, false>, grid, block, 0, st, a, k);
-  return vec ? launch_pdl(k_accept_sample<1, true>, grid, block, 0, st, a, k)
-             : launch_pdl(k_accept_sample<1, false>, grid, block, 0, st, a, k);
+  return launch_pdl(accept_kernel(dtype, vec, a.K), dim3(a.P, a.B), dim3(kThreads), 0, st, a, k);
 }
 
 }  // namespace specv
