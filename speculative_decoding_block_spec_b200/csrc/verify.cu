@@ -73,7 +73,8 @@ __global__ void __launch_bounds__(kThreads, 3) k_accept_sample(VerifyArgs a, flo
   __shared__ int s_x[kMaxL];
   __shared__ float s_u[kMaxL], s_w[kMaxK];
   __shared__ float s_c[kMaxK + 1], s_mm[kMaxK + 1];
-  __shared__ int s_flags, s_j, s_last, s_fail;
+  __shared__ int s_flags, s_j, s_last, s_fail, s_scan;
+  __shared__ Best s_best[kWarps];
   __shared__ int s_cnt[2 * kWarps];
 
   const int b = blockIdx.y, p = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
@@ -250,9 +251,11 @@ __global__ void __launch_bounds__(kThreads, 3) k_accept_sample(VerifyArgs a, flo
         }
 #pragma unroll
         for (int e = 0; e < E; ++e) {
-          const Best c{static_cast<double>(xt[e]) * invT + static_cast<double>(gv[e]), static_cast<int>(u * E + e)};
-          if (c.score > bb.score) bb = c;
           q[e] = 0.f;
+          if (!resid) {  // bonus draw (after a rejection the bonus rule is only a rare fallback, below)
+            const Best c{static_cast<double>(xt[e]) * invT + static_cast<double>(gv[e]), static_cast<int>(u * E + e)};
+            if (c.score > bb.score) bb = c;
+          }
         }
         if (resid) {
 #pragma unroll
@@ -314,18 +317,45 @@ __global__ void __launch_bounds__(kThreads, 3) k_accept_sample(VerifyArgs a, flo
   __syncthreads();
   if (!s_last) return;
   if (tid == 0) {
+    s_scan = 0;
     if (flags == 0) {
       const int j = s_j;
       const unsigned long long kr = __ldcg(a.keys + 2 * b), kb = __ldcg(a.keys + 2 * b + 1);
-      const int term = (j < ell && kr) ? key_token(kr) : key_token(kb);
-      if (term >= 0) out[j] = term;
-      else s_fail = 1;
+      if (j < ell && !kr) {
+        s_scan = 1;  // rounding left no p > q after a rejection: bonus rule on row j, below
+      } else {
+        const int term = j < ell ? key_token(kr) : key_token(kb);
+        if (term >= 0) out[j] = term;
+        else s_fail = 1;
+      }
     }
     a.keys[2 * b] = 0ull;
     a.keys[2 * b + 1] = 0ull;
     a.tickets[b] = 0;
   }
   __syncthreads();
+  if (s_scan) {  // rare: this block takes argmax_v x_j(v) / T + g(v) over the whole row
+    const int j = s_j;
+    const double invT = 1.0 / static_cast<double>(a.T);
+    const char* trow = static_cast<const char*>(a.target) + (toff + j) * V * Elem<DT>::kBytes;
+    const float* grow = a.g + (static_cast<int64_t>(b) * (L + 1) + j) * V;
+    Best bb{-INFINITY, -1};
+    for (int64_t v = tid; v < V; v += kThreads) {
+      const Best c{static_cast<double>(Elem<DT>::at(trow, v)) * invT + static_cast<double>(__ldg(grow + v)),
+                   static_cast<int>(v)};
+      if (c.score > bb.score) bb = c;
+    }
+    warp_best(bb);
+    if (lane == 0) s_best[tid >> 5] = bb;
+    __syncthreads();
+    if (tid == 0) {
+      Best t = s_best[0];
+      for (int w = 1; w < kWarps; ++w) best_merge(t, s_best[w]);
+      if (t.idx >= 0) out[j] = t.idx;
+      else s_fail = 1;
+    }
+    __syncthreads();
+  }
   if (s_fail) {  // no finite candidate in the terminal row: the request fails as a whole
     for (int i = tid; i <= L; i += kThreads) out[i] = -1;
     if (tid == 0) {

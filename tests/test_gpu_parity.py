@@ -157,6 +157,40 @@ def test_q_equals_p_accepts_everything():
     check_verify(_cpu(acc), _cpu(out), ref, verify_len=vl)
 
 
+def test_rejection_with_empty_residual_draws_row_j_by_the_bonus_rule():
+    """Speculative sampling with rejection correction ("DBLAST", Pith review,
+    "Assumptions"): after a rejection the residual max(0, p - q) has positive
+    mass in exact arithmetic. Here target and draft rows are all zero except
+    at the drafted token, which sits at -200 in the target and -199 in the
+    draft: the test rejects (rho = exp(-1)), but that token's share of either
+    normaliser is below the precision of the sum, and every other term is
+    exactly 1, so both normalisers are exactly V - 1 in any summation order,
+    fp32 and fp64 alike, and no element has p > q. Both sides then draw row j
+    by the bonus rule, which on the GPU is the request's last block scanning
+    the row."""
+    rng = np.random.default_rng(41)
+    B, L, V = 3, 4, 151936
+    tt = np.zeros((B, L + 1, V), np.uint16)  # bf16 zeros
+    tokens = rng.integers(0, V, (B, L)).astype(np.int32)
+    for b in range(B):
+        for i in range(L):
+            tt[b, i, tokens[b, i]] = 0xC348  # -200.0
+    dd = tt[:, :L].copy()
+    for b in range(B):
+        for i in range(L):
+            dd[b, i, tokens[b, i]] = 0xC347  # -199.0
+    u = np.full((B, L), 0.99, np.float32)
+    g = synth.gumbel(rng, (B, L + 1, V)).astype(np.float32)
+    ref = oracle.verify(tt, dd, tokens, u, g, 1.0, n_threads=NT, diag=True)
+    np.testing.assert_array_equal(ref["accept_len"], np.zeros(B, np.int32))
+    ws = specv.Workspace(specv.verify_workspace_size(B, L, 1, V))
+    acc, out = specv.spec_verify_block(logits_to_torch(tt), logits_to_torch(dd), torch.from_numpy(tokens).cuda(),
+                                       torch.from_numpy(u).cuda(), torch.from_numpy(g).cuda(), 1.0, workspace=ws)
+    np.testing.assert_array_equal(_cpu(acc), ref["accept_len"])
+    np.testing.assert_array_equal(_cpu(out), ref["out_tokens"])
+    assert ws.status() == 0
+
+
 def test_one_hot_target_and_vocab_edge_tokens():
     rng = np.random.default_rng(13)
     B, L, V = 4, 6, 151936
