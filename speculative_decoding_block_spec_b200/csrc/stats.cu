@@ -6,14 +6,17 @@
 // Drafting for Stochastic Speculative Decoding", Pith review, "Assumptions";
 // target sampling at T = 1.5 in "What would settle it").
 //
-// Design. A persistent grid of G blocks (a multiple of the SM count) splits
-// the flattened units of every row evenly, so every block streams the same
-// number of bytes whatever the row count; a block's range covers a tail of
-// one row, whole rows, and a head of another. Each thread keeps an online
-// (max, sum of 2^((x - max) log2e / T)) over its 16-byte vectors: a group of
-// U vectors is loaded at once, its maximum taken exactly on the raw bf16
-// pairs, then one exponential per element. Blocks write one partial per
-// (row, block); consumers merge the few partials of a row.
+// Design. A grid of G blocks splits the flattened 16-byte units of every row
+// evenly, so every block streams the same number of bytes whatever the row
+// count; a block's range covers a tail of one row, whole rows, and a head of
+// another. Each thread keeps an online (max, sum of 2^((x - max) log2e / T))
+// over its vectors: a group is loaded at once, its maximum taken exactly on
+// the raw bf16 pairs, then one exponential per element. Blocks write one
+// partial per (row, block); consumers merge the few partials of a row. Two
+// kernels share this split: k_row_stats (several blocks per SM, each thread
+// striding its block's range) and k_row_stats_dyn (one block per SM whose
+// warps take row-aligned slices of the range from a shared counter, for
+// windows of at most 256 MB).
 #include <algorithm>
 #include <mutex>
 

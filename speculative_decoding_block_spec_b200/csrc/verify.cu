@@ -18,12 +18,16 @@
 //   2. take the accept decisions in one warp (decide_warp), identically in
 //      every block, so no block waits for another; block 0 then writes the
 //      accepted length and every output token but the terminal one;
-//   3. score 1/P of terminal row j (target, K draft rows, Gumbel row) and
-//      publish each warp's best residual and bonus candidates as 64-bit
-//      order-preserving keys with red.max (no return, no wait).
+//   3. score 1/P of terminal row j and publish each warp's best candidate as
+//      a 64-bit order-preserving key with red.max (no return, no wait): after
+//      a rejection the residual log(p - q) + g from the target, K draft and
+//      Gumbel rows; with none, the bonus x / T + g from the target and Gumbel
+//      rows.
 // The last of the request's blocks to finish (per-request atomic ticket)
 // writes the terminal token and clears the request's keys and ticket, so the
-// workspace is ready for the next call.
+// workspace is ready for the next call. If rounding left no element with
+// p > q after a rejection (impossible in exact arithmetic), that block draws
+// row j by the bonus rule itself.
 #include <algorithm>
 
 #include "common.cuh"
