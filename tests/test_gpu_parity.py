@@ -133,6 +133,24 @@ def test_seed_sweep_block_and_mixture(seed, path):
     check_verify(_cpu(acc), _cpu(out), ref, verify_len=vl)
 
 
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("K,L,V,dtype", [(5, 16, 32768, "bf16"), (8, 32, 8192, "bf16"), (8, 7, 1001, "f32")])
+def test_mixture_beyond_one_draft_batch_and_largest_shapes(K, L, V, dtype, path):
+    """Latent-mixture drafts ("DBLAST", "What carries the argument", Eq. 5)
+    with more categories than one batch of terminal draft loads (K > 4), up to
+    the largest K = 8 and L = 32, on the vector and the scalar path."""
+    x = synth.custom(B=6, L=L, V=V, K=K, T=1.1, dtype=dtype, n_peaks=4, peak=5.0, draft_sigma=0.6, seed=K + L,
+                     cid=400 + K + L)
+    vl = np.random.default_rng(K * L).integers(0, L + 1, size=6).astype(np.int32)
+    vl[0] = L
+    ref = oracle.verify(x.target, x.draft, x.tokens, x.u, x.g, x.w.T, mix_w=x.mix_w, verify_len=vl,
+                        n_threads=NT, diag=True)
+    assert np.any(ref["accept_len"] < vl)  # some request rejects: the residual over K draft rows is exercised
+    d = to_torch(x)
+    acc, out = _verify(d, x, x.w.T, verify_len=torch.from_numpy(vl).cuda(), path=path)
+    check_verify(_cpu(acc), _cpu(out), ref, verify_len=vl)
+
+
 # -------------------------------------------------------------- identities
 
 def test_k1_mixture_is_bit_identical_to_block():
