@@ -22,6 +22,8 @@ struct DecideIn {
   const float* xg;   // raw logit at the drafted token, per row
   const float* m;    // row max of raw logits
   const float* s;    // sum 2^((x - m) log2e / T)
+  const double* ls;  // log(s) in fp64, per row (read when K > 1)
+  const double* lw;  // log q(z|y) in fp64 [K], nullptr for w = 1 (K == 1)
   const int* x;      // drafted tokens [ell]
   int ell, K, L;
   float T;
@@ -35,15 +37,18 @@ struct DecideOut {
   float cz[kMaxK], mz[kMaxK];
 };
 
-// Run by the 32 lanes of one warp (lane i tests position i). A fast fp32
-// pass computes every ratio rho_i; only when some tested lane lies close to
-// its threshold (|u_i - min(1, rho_i)| below 1e-5 for independent drafts,
-// 2e-4 with a posterior, i.e. 10x the fp32 error) or meets a non-finite value
-// does the warp redo the decisions in fp64, where the normalisers are the
-// only fp32 quantities. u, mix_w: this request's rows.
-__device__ __forceinline__ DecideOut decide_warp_fp64(const DecideIn& in, const float* u, const float* mix_w);
+// Run by the 32 lanes of one warp (lane i tests position i). A fast pass
+// computes every ratio rho_i: for independent drafts in fp32 from the raw
+// logit differences; with a posterior, the per-position log-probabilities
+// and their prefix sums in fp64 (from fp64 log-normalisers) and only the
+// K-way log-sum-exps and the final exponential in fp32. Its error in rho is
+// below 1e-6 relative; only when some tested lane lies within 1e-5 of its
+// threshold |u_i - min(1, rho_i)| or meets a non-finite value does the warp
+// redo the decisions fully in fp64, where the normalisers are the only fp32
+// quantities. u: this request's uniforms.
+__device__ __forceinline__ DecideOut decide_warp_fp64(const DecideIn& in, const float* u);
 
-__device__ __forceinline__ DecideOut decide_warp(const DecideIn& in, const float* u, const float* mix_w) {
+__device__ __forceinline__ DecideOut decide_warp(const DecideIn& in, const float* u) {
   const int lane = threadIdx.x & 31;
   const int ell = in.ell, K = in.K;
   const bool act = lane < ell;
@@ -62,52 +67,55 @@ __device__ __forceinline__ DecideOut decide_warp(const DecideIn& in, const float
       finite = isfinite(d) && isfinite(in.xg[q]) && isfinite(in.xg[lane]);
     }
   } else {
-    float lqz[kMaxK], amax = -INFINITY;
+    const double invTd = 1.0 / static_cast<double>(in.T);
+    double lqz[kMaxK], lpd[kMaxK], amax = -INFINITY;
 #pragma unroll
     for (int z = 0; z < kMaxK; ++z) {
-      lqz[z] = 0.f;
+      lqz[z] = 0.0;
+      lpd[z] = 0.0;
       if (z < K) {
         if (act) {
           const int q = ell + z * ell + lane;
-          lqz[z] = (in.xg[q] - in.m[q]) * invT - logf(in.s[q]);
+          lqz[z] = static_cast<double>(in.xg[q] - in.m[q]) * invTd - in.ls[q];  // x - m is exact in fp32
         }
-        float v = __shfl_up_sync(0xffffffffu, lqz[z], 1);
-        if (lane == 0) v = 0.f;
+        double v = __shfl_up_sync(0xffffffffu, lqz[z], 1);
+        if (lane == 0) v = 0.0;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-          const float t = __shfl_up_sync(0xffffffffu, v, o);
+          const double t = __shfl_up_sync(0xffffffffu, v, o);
           if (lane >= o) v += t;
         }
-        lpi[z] = (mix_w ? logf(mix_w[z]) : 0.f) + v;
-        amax = fmaxf(amax, lpi[z]);
+        lpd[z] = (in.lw ? in.lw[z] : 0.0) + v;
+        amax = fmax(amax, lpd[z]);
       }
     }
     float sa = 0.f;
 #pragma unroll
     for (int z = 0; z < kMaxK; ++z)
-      if (z < K) sa += expf(lpi[z] - amax);
-    const float norm = amax + logf(sa);
-    float tmax = -INFINITY;
+      if (z < K) sa += expf(static_cast<float>(lpd[z] - amax));
+    const double norm = amax + static_cast<double>(logf(sa));
+    double tmax = -INFINITY;
 #pragma unroll
     for (int z = 0; z < kMaxK; ++z) {
       if (z < K) {
-        lpi[z] -= norm;
-        tmax = fmaxf(tmax, lpi[z] + lqz[z]);
+        lpd[z] -= norm;
+        lpi[z] = static_cast<float>(lpd[z]);
+        tmax = fmax(tmax, lpd[z] + lqz[z]);
       }
     }
     float st = 0.f;
 #pragma unroll
     for (int z = 0; z < kMaxK; ++z)
-      if (z < K) st += expf(lpi[z] + lqz[z] - tmax);
-    const float lq = tmax + logf(st);
-    const float lp = act ? (in.xg[lane] - in.m[lane]) * invT - logf(in.s[lane]) : 0.f;
-    rho = expf(lp - lq);
+      if (z < K) st += expf(static_cast<float>(lpd[z] + lqz[z] - tmax));
+    const double lq = tmax + static_cast<double>(logf(st));
+    const double lp = act ? static_cast<double>(in.xg[lane] - in.m[lane]) * invTd - in.ls[lane] : 0.0;
+    rho = expf(static_cast<float>(lp - lq));
     finite = isfinite(norm) && isfinite(lp) && isfinite(lq);
   }
   const float thr = fminf(1.f, rho);
-  const float band = K == 1 ? 1e-5f : 2e-4f;
+  constexpr float band = 1e-5f;
   const bool close = act && (!finite || isnan(rho) || fabsf(uu - thr) < band);
-  if (__any_sync(0xffffffffu, close)) return decide_warp_fp64(in, u, mix_w);
+  if (__any_sync(0xffffffffu, close)) return decide_warp_fp64(in, u);
   const unsigned stop = __ballot_sync(0xffffffffu, act && !(uu < thr));
   DecideOut o;
   o.j = stop ? __ffs(stop) - 1 : ell;
@@ -135,7 +143,7 @@ __device__ __forceinline__ DecideOut decide_warp(const DecideIn& in, const float
   return o;
 }
 
-__device__ __forceinline__ DecideOut decide_warp_fp64(const DecideIn& in, const float* u, const float* mix_w) {
+__device__ __forceinline__ DecideOut decide_warp_fp64(const DecideIn& in, const float* u) {
   const int lane = threadIdx.x & 31;
   const int ell = in.ell, K = in.K;
   const double T = static_cast<double>(in.T);
@@ -170,7 +178,7 @@ __device__ __forceinline__ DecideOut decide_warp_fp64(const DecideIn& in, const 
         const double t = __shfl_up_sync(0xffffffffu, v, o);
         if (lane >= o) v += t;
       }
-      const double lw = mix_w ? log(static_cast<double>(mix_w[z])) : 0.0;
+      const double lw = in.lw ? in.lw[z] : 0.0;
       lpi[z] = lw + v;
       amax = fmax(amax, lpi[z]);
     }

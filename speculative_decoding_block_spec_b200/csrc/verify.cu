@@ -75,7 +75,8 @@ __global__ void __launch_bounds__(kThreads, 3) k_accept_sample(VerifyArgs a, flo
   __shared__ float s_xg[kMaxRows];  // logit at the drafted token, per request row
   __shared__ float s_m[kMaxRows], s_s[kMaxRows];
   __shared__ int s_x[kMaxL];
-  __shared__ float s_u[kMaxL], s_w[kMaxK];
+  __shared__ float s_u[kMaxL];
+  __shared__ double s_lw[kMaxK], s_ls[kMaxRows];
   __shared__ float s_c[kMaxK + 1], s_mm[kMaxK + 1];
   __shared__ int s_flags, s_j, s_last, s_fail, s_scan;
   __shared__ Best s_best[kWarps];
@@ -128,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_accept_sample(VerifyArgs a, flo
     s_x[tid] = x;
     s_u[tid] = a.u[static_cast<int64_t>(b) * L + tid];
   }
-  if (tid < K && a.mix_w) s_w[tid] = a.mix_w[static_cast<int64_t>(b) * K + tid];
+  if (tid < K && a.mix_w) s_lw[tid] = log(static_cast<double>(a.mix_w[static_cast<int64_t>(b) * K + tid]));
 
   pdl_wait();
   pdl_trigger();
@@ -156,6 +157,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_accept_sample(VerifyArgs a, flo
     s_m[q] = m;
     s_s[q] = s;
     s_xg[q] = xq;
+    if (K > 1) s_ls[q] = log(static_cast<double>(s));
     if (!isfinite(m) || !isfinite(s)) atomicOr(&s_flags, kFlagNonFinite);
   }
   __syncthreads();
@@ -165,8 +167,8 @@ __global__ void __launch_bounds__(kThreads, 3) k_accept_sample(VerifyArgs a, flo
   if (tid < 32) {
     int j = ell, f = s_flags;
     if (f == 0) {
-      const DecideIn in{s_xg, s_m, s_s, s_x, ell, K, L, a.T};
-      const DecideOut o = decide_warp(in, s_u, a.mix_w ? s_w : nullptr);
+      const DecideIn in{s_xg, s_m, s_s, s_ls, a.mix_w ? s_lw : nullptr, s_x, ell, K, L, a.T};
+      const DecideOut o = decide_warp(in, s_u);
       j = o.j;
       if (o.bad) f |= kFlagNonFinite;
       if (lane == 0) {
