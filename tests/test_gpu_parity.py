@@ -151,6 +151,42 @@ def test_mixture_beyond_one_draft_batch_and_largest_shapes(K, L, V, dtype, path)
     check_verify(_cpu(acc), _cpu(out), ref, verify_len=vl)
 
 
+@pytest.mark.parametrize("K", [1, 2])
+def test_largest_batch(K):
+    """B = SPEC_MAX_B requests (one sampling block each) with ragged verify lengths."""
+    B, L, V = 4096, 2, 256
+    x = synth.custom(B=B, L=L, V=V, K=K, T=1.0, dtype="bf16", n_peaks=2, peak=3.0, draft_sigma=0.5, seed=50 + K,
+                     cid=450 + K)
+    vl = np.random.default_rng(50 + K).integers(0, L + 1, size=B).astype(np.int32)
+    ref = oracle.verify(x.target, x.draft, x.tokens, x.u, x.g, 1.0, mix_w=x.mix_w, verify_len=vl, n_threads=NT,
+                        diag=True)
+    d = to_torch(x)
+    acc, out = _verify(d, x, 1.0, verify_len=torch.from_numpy(vl).cuda())
+    check_verify(_cpu(acc), _cpu(out), ref, verify_len=vl)
+
+
+def test_largest_vocabulary_and_top_token_index():
+    """V = SPEC_MAX_V = 2^20: the terminal keys carry the token in 20 bits, so
+    the draws land on tokens V - 1 (bonus row) and V - 2 (residual)."""
+    B, L, V = 2, 2, 1 << 20
+    rng = np.random.default_rng(60)
+    t = rng.standard_normal((B, L + 1, V)).astype(np.float32)
+    dr = t[:, :L].copy()
+    tokens = np.array([[3, 5], [7, 9]], np.int32)
+    t[0, L, V - 1] = 60.0        # request 0 accepts both positions (draft == target): bonus row peaks at V - 1
+    t[1, 0, V - 2] = 60.0        # request 1: target row 0 peaks at V - 2, which the draft lacks, so x_0 is
+    dr[1, 0, tokens[1, 0]] = 40.0  # rejected (the draft is confident in it) and the residual is V - 2
+    tt, dd = f32_to_bf16_bits(t), f32_to_bf16_bits(dr)
+    u = np.full((B, L), 0.5, np.float32)
+    g = synth.gumbel(rng, (B, L + 1, V)).astype(np.float32)
+    ref = oracle.verify(tt, dd, tokens, u, g, 1.0, n_threads=NT, diag=True)
+    np.testing.assert_array_equal(ref["accept_len"], [2, 0])
+    assert ref["out_tokens"][0, 2] == V - 1 and ref["out_tokens"][1, 0] == V - 2
+    acc, out = specv.spec_verify_block(logits_to_torch(tt), logits_to_torch(dd), torch.from_numpy(tokens).cuda(),
+                                       torch.from_numpy(u).cuda(), torch.from_numpy(g).cuda(), 1.0)
+    check_verify(_cpu(acc), _cpu(out), ref)
+
+
 # -------------------------------------------------------------- identities
 
 def test_k1_mixture_is_bit_identical_to_block():
