@@ -262,6 +262,34 @@ def test_zero_verify_length_is_a_bonus_draw():
     assert np.all(r["out_tokens"][:, 1:] == -1)
 
 
+def test_rejection_with_empty_residual_uses_the_bonus_rule_on_row_j():
+    """After a rejection the residual max(0, p - q) is empty only through
+    rounding: here target and draft rows are all zero except the drafted
+    token (-200 in the target, -199 in the draft), so the test rejects
+    (rho = exp(-1) < u = 0.99) while both normalisers are exactly V - 1 and
+    p == q everywhere else. The reading taken: row j is then drawn by the
+    bonus rule, argmax_v x_j(v) / T + g[b, j, v]."""
+    B, L, V = 2, 3, 50
+    rng = np.random.default_rng(8)
+    target = np.zeros((B, L + 1, V), np.float32)
+    tokens = rng.integers(0, V, (B, L)).astype(np.int32)
+    for b in range(B):
+        for i in range(L):
+            target[b, i, tokens[b, i]] = -200.0
+    draft = target[:, :L].copy()
+    for b in range(B):
+        for i in range(L):
+            draft[b, i, tokens[b, i]] = -199.0
+    u = np.full((B, L), 0.99, np.float32)
+    g = synth.gumbel(rng, (B, L + 1, V)).astype(np.float32)
+    r = oracle.verify(target, draft, tokens, u, g, 1.0, diag=True)
+    np.testing.assert_array_equal(r["accept_len"], 0)
+    np.testing.assert_allclose(r["rho"][:, 0], math.exp(-1.0), rtol=1e-12)
+    expect = (target[:, 0].astype(np.float64) + g[:, 0].astype(np.float64)).argmax(axis=1)
+    np.testing.assert_array_equal(r["out_tokens"][:, 0], expect)
+    assert np.all(r["out_tokens"][:, 1:] == -1)
+
+
 def test_device_style_error_flags():
     x = synth.custom(B=3, L=4, V=64, dtype="f32", seed=4)
     tok = x.tokens.copy()
