@@ -67,8 +67,9 @@ def test_softmax_parity(rows, V, dtype, T, probs):
 
 def _verify(d, x, T, verify_len=None, target=None, row_off=None, path="fused"):
     """One verification through the C ABI. path 'fused' is the public one-call
-    entry point (one persistent kernel when the shapes allow it); 'split' runs
-    its two stages, spec_verify_window_stats then spec_verify_accept."""
+    entry point (spec_verify_block / spec_verify_mixture, which launch both
+    stages chained); 'split' makes the two stage calls itself,
+    spec_verify_window_stats then spec_verify_accept."""
     tgt = d["target"] if target is None else target
     mix = d.get("mix_w") if x.w.K > 1 else None
     if path == "split":
