@@ -63,6 +63,47 @@ def test_softmax_parity(rows, V, dtype, T, probs):
         np.testing.assert_allclose(_cpu(got[2]), ref[2], rtol=1e-5, atol=1e-37)
 
 
+@pytest.mark.parametrize("dtype,V,stride", [("bf16", 4000, 4096), ("bf16", 4000, 4003), ("f32", 1000, 1024)])
+def test_softmax_padded_row_stride(dtype, V, stride):
+    """Rows start every `stride` elements and only their first V are logits
+    (row_stride > V in the C ABI); the padding holds values that would
+    dominate every row if it were read. 4096 keeps the 16-byte path, 4003
+    forces the scalar one."""
+    rows, T = 37, 1.3
+    rng = np.random.default_rng(stride + V)
+    full = rng.standard_normal((rows, stride)).astype(np.float32) * 2
+    full[:, V:] = 1.0e4
+    xs = f32_to_bf16_bits(full) if dtype == "bf16" else full
+    ref = oracle.softmax_T(np.ascontiguousarray(xs[:, :V]), T, probs=True)
+    logits = logits_to_torch(xs)
+    rmax = torch.empty(rows, dtype=torch.float32, device="cuda")
+    rlse = torch.empty_like(rmax)
+    probs = torch.empty((rows, V), dtype=torch.float32, device="cuda")
+    ws = specv.Workspace(specv.softmax_workspace_size(rows))
+    st = specv.lib().spec_softmax_T(logits.data_ptr(), 1 if dtype == "bf16" else 0, rows, V, stride, T,
+                                    rmax.data_ptr(), rlse.data_ptr(), probs.data_ptr(), ws.ptr(), ws.nbytes,
+                                    torch.cuda.current_stream().cuda_stream)
+    assert st == 0
+    np.testing.assert_allclose(_cpu(rmax), ref[0], rtol=1e-5, atol=0)
+    np.testing.assert_allclose(_cpu(rlse), ref[1], rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(_cpu(probs), ref[2], rtol=1e-5, atol=1e-37)
+
+
+@pytest.mark.parametrize("K", [1, 3])
+@pytest.mark.parametrize("T", [0.3, 3.0])
+def test_extreme_temperatures(T, K):
+    """Sharp (T = 0.3: logits / T reach about 30) and flat (T = 3) target and
+    draft distributions, same T for both ("DBLAST", "Assumptions")."""
+    x = synth.custom(B=6, L=12, V=65536, K=K, T=T, dtype="bf16", n_peaks=8, peak=6.0, draft_sigma=0.7,
+                     seed=int(T * 10) + K, cid=480 + int(T * 10) + K)
+    vl = np.random.default_rng(int(T * 10) + K).integers(0, 13, size=6).astype(np.int32)
+    ref = oracle.verify(x.target, x.draft, x.tokens, x.u, x.g, T, mix_w=x.mix_w, verify_len=vl, n_threads=NT,
+                        diag=True)
+    d = to_torch(x)
+    acc, out = _verify(d, x, T, verify_len=torch.from_numpy(vl).cuda())
+    check_verify(_cpu(acc), _cpu(out), ref, verify_len=vl)
+
+
 # ------------------------------------------------------------ the workloads
 
 def _verify(d, x, T, verify_len=None, target=None, row_off=None, path="fused"):
