@@ -24,7 +24,7 @@ def _load():
         lib = ctypes.CDLL(build_oracle())
         P, I, I64, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
         lib.oracle_softmax_T.argtypes = [P, I, I64, I64, I64, D, P, P, P]
-        lib.oracle_verify.argtypes = [P, P, P, I, P, P, P, P, P, I, I, I, I64, D, I, P, P, P]
+        lib.oracle_verify.argtypes = [P, P, P, I, P, P, P, P, P, I, I, I, I64, D, D, I, P, P, P]
         lib.oracle_dvl_allocate.argtypes = [P, I, I, I, P, P, P, P]
         lib.oracle_pack.argtypes = [P, I, I, I, I64, P, P, P]
         for f in (lib.oracle_softmax_T, lib.oracle_verify, lib.oracle_dvl_allocate, lib.oracle_pack):
@@ -69,11 +69,12 @@ def softmax_T(x, T, probs=False):
 
 
 def verify(target, draft, tokens, u, g, T, *, mix_w=None, verify_len=None, target_row_off=None,
-           n_threads=1, diag=False):
+           n_threads=1, diag=False, top_p=1.0):
     """Speculative verification of B drafted blocks (see oracle.h).
 
     target: [B, L+1, V] dense, or packed [S, V] with target_row_off [B].
     draft:  [B, L, V] (independent) or [B, K, L, V] (latent mixture, with mix_w [B, K]).
+    top_p:  nucleus filter of every target and draft row (1 = none; see oracle.h).
     Returns dict(accept_len, out_tokens, flags[, diagnostics...])."""
     target, dt = _logits(target)
     draft, dt2 = _logits(draft)
@@ -104,7 +105,7 @@ def verify(target, draft, tokens, u, g, T, *, mix_w=None, verify_len=None, targe
                    argmax_kappa=np.empty(B), terminal_dist=np.empty((B, V)))
         dptr = ctypes.byref(_Diag(*[_ptr(res[f[0]]) for f in _Diag._fields_]))
     st = _load().oracle_verify(_ptr(target), _ptr(off), _ptr(draft), dt, _ptr(tokens), _ptr(vl),
-                               _ptr(u), _ptr(g), _ptr(w), K, B, L, V, float(T), int(n_threads),
+                               _ptr(u), _ptr(g), _ptr(w), K, B, L, V, float(T), float(top_p), int(n_threads),
                                _ptr(acc), _ptr(out), dptr)
     if st < 0:
         raise ValueError("oracle_verify rejected its arguments (%d)" % st)

@@ -84,6 +84,63 @@ static double logsumexp(const double* a, int n) {
   return m + log(s);
 }
 
+/* Top-p (nucleus) filtering of one temperature-softmax row: the sampling
+ * filter of target sampling (DBLAST review, "What would settle it":
+ * temperature 1.5 with top-p 0.95; "Assumptions": target probabilities are
+ * taken under the same sampling filter). The nucleus is the shortest prefix
+ * of the tokens ordered by probability (descending, ties to the lower index)
+ * whose mass reaches top_p; filtered log-probabilities are log p(v) minus the
+ * log of that mass inside it and -inf outside. A nucleus is kept as its last
+ * member (log-probability, token) and the log of its mass. */
+typedef struct {
+  int all;          /* top_p >= 1: no filtering */
+  double lp_cut;    /* log-probability of the last member */
+  int64_t v_cut;    /* its token; equal log-probabilities are members up to it */
+  double log_mass;  /* log of the nucleus mass */
+} nucleus;
+
+typedef struct { double lp; int64_t v; } ranked;
+
+static int ranked_order(const void* pa, const void* pb) {
+  const ranked* a = (const ranked*)pa;
+  const ranked* b = (const ranked*)pb;
+  if (a->lp > b->lp) return -1;
+  if (a->lp < b->lp) return 1;
+  return (a->v > b->v) - (a->v < b->v);
+}
+
+static void row_nucleus(const void* row, int dtype, int64_t V, double T, double lse, double top_p, nucleus* n) {
+  n->all = top_p >= 1.0;
+  n->lp_cut = -INFINITY;
+  n->v_cut = V - 1;
+  n->log_mass = 0.0;
+  if (n->all) return;
+  ranked* r = malloc((size_t)V * sizeof(ranked));
+  for (int64_t v = 0; v < V; ++v) {
+    r[v].lp = load_x(row, dtype, v) / T - lse;
+    r[v].v = v;
+  }
+  qsort(r, (size_t)V, sizeof(ranked), ranked_order);
+  double mass = 0.0;
+  int64_t k = 0;
+  for (; k < V; ++k) {
+    mass += exp(r[k].lp);
+    if (mass >= top_p) break;
+  }
+  if (k == V) k = V - 1; /* rounding kept the total just below top_p: the whole row */
+  n->lp_cut = r[k].lp;
+  n->v_cut = r[k].v;
+  n->log_mass = log(mass);
+  free(r);
+}
+
+/* Filtered log-probability of token v whose unfiltered one is lpv. */
+static double nucleus_lp(const nucleus* n, double lpv, int64_t v) {
+  if (n->all) return lpv;
+  const int in = lpv > n->lp_cut || (lpv == n->lp_cut && v <= n->v_cut);
+  return in ? lpv - n->log_mass : -INFINITY;
+}
+
 typedef struct {
   const void* target;
   const int32_t* target_row_off;
@@ -97,6 +154,7 @@ typedef struct {
   int K, B, L;
   int64_t V;
   double T;
+  double top_p;
   int32_t* accept_len;
   int32_t* out_tokens;
   const oracle_diag* diag;
@@ -172,10 +230,13 @@ static int verify_one(const verify_args* a, int b) {
   double* s1 = calloc((size_t)K, sizeof(double));
   double* s2 = calloc((size_t)K, sizeof(double));
   double* lqv = calloc((size_t)K, sizeof(double));
+  nucleus* nt = calloc((size_t)L + 1, sizeof(nucleus));       /* target rows 0..ell */
+  nucleus* nd = calloc((size_t)K * L + 1, sizeof(nucleus));   /* draft rows (z, i) */
   double* dist = d && d->terminal_dist ? d->terminal_dist + (int64_t)b * V : NULL;
   double m_unused;
 
-  /* Step 1: temperature softmax normalisers of every tested row. */
+  /* Step 1: temperature softmax normalisers (and, below top_p = 1, nuclei) of
+   * every tested row. */
   for (int i = 0; i < ell; ++i) {
     row_softmax_stats(trow[i], a->dtype, V, T, &m_unused, &lse_t[i]);
     if (!isfinite(lse_t[i]) || !isfinite(m_unused)) flags |= ORC_FLAG_NONFINITE;
@@ -185,12 +246,16 @@ static int verify_one(const verify_args* a, int b) {
     }
   }
   if (flags) goto done;
-
-  /* Step 2: log-probabilities of the drafted tokens under target and branches. */
   for (int i = 0; i < ell; ++i) {
-    lp[i] = load_x(trow[i], a->dtype, x[i]) / T - lse_t[i];
+    row_nucleus(trow[i], a->dtype, V, T, lse_t[i], a->top_p, &nt[i]);
+    for (int z = 0; z < K; ++z) row_nucleus(DROW(z, i), a->dtype, V, T, lse_d[z * L + i], a->top_p, &nd[z * L + i]);
+  }
+
+  /* Step 2: (filtered) log-probabilities of the drafted tokens under target and branches. */
+  for (int i = 0; i < ell; ++i) {
+    lp[i] = nucleus_lp(&nt[i], load_x(trow[i], a->dtype, x[i]) / T - lse_t[i], x[i]);
     for (int z = 0; z < K; ++z)
-      lqz[z * L + i] = load_x(DROW(z, i), a->dtype, x[i]) / T - lse_d[z * L + i];
+      lqz[z * L + i] = nucleus_lp(&nd[z * L + i], load_x(DROW(z, i), a->dtype, x[i]) / T - lse_d[z * L + i], x[i]);
   }
   for (int z = 0; z < K; ++z) logw[z] = a->mix_w ? log((double)a->mix_w[(int64_t)b * K + z]) : 0.0;
 
@@ -203,7 +268,9 @@ static int verify_one(const verify_args* a, int b) {
     if ((flags |= category_posterior(logw, lqz, K, L, i, logpi, s1))) goto done;
     for (int z = 0; z < K; ++z) lqv[z] = lqz[z * L + i];
     const double lq = proposal_logprob(logpi, lqv, K, s2);
-    const double rho = exp(lp[i] - lq);
+    /* A token outside the filtered target has p = 0, so rho = 0 (even when the
+     * filtered proposal gives it 0 as well). */
+    const double rho = (lp[i] == -INFINITY && a->top_p < 1.0) ? 0.0 : exp(lp[i] - lq);
     if (isnan(rho)) { flags |= ORC_FLAG_NONFINITE; goto done; }
     const double thr = rho < 1.0 ? rho : 1.0;
     const double ui = (double)a->u[(int64_t)b * L + i];
@@ -229,9 +296,9 @@ static int verify_one(const verify_args* a, int b) {
     if ((flags |= category_posterior(logw, lqz, K, L, j, logpi, s1))) goto done;
     double rsum = 0.0;
     for (int64_t v = 0; v < V; ++v) {
-      const double lpv = load_x(trow[j], a->dtype, v) / T - lse_t[j];
+      const double lpv = nucleus_lp(&nt[j], load_x(trow[j], a->dtype, v) / T - lse_t[j], v);
       for (int z = 0; z < K; ++z)
-        lqv[z] = load_x(DROW(z, j), a->dtype, v) / T - lse_d[z * L + j];
+        lqv[z] = nucleus_lp(&nd[z * L + j], load_x(DROW(z, j), a->dtype, v) / T - lse_d[z * L + j], v);
       const double lqv_mix = proposal_logprob(logpi, lqv, K, s2);
       const double pv = exp(lpv), qv = exp(lqv_mix);
       const double r = pv - qv;
@@ -256,12 +323,13 @@ static int verify_one(const verify_args* a, int b) {
     if (j == ell) {
       row_softmax_stats(trow[ell], a->dtype, V, T, &m_unused, &lse);
       if (!isfinite(lse) || !isfinite(m_unused)) { flags |= ORC_FLAG_NONFINITE; goto done; }
+      row_nucleus(trow[ell], a->dtype, V, T, lse, a->top_p, &nt[ell]);
     } else {
       lse = lse_t[j];
     }
     best1 = best2 = -INFINITY; kap1 = kap2 = 1.0; t = -1;
     for (int64_t v = 0; v < V; ++v) {
-      const double lpv = load_x(trow[j], a->dtype, v) / T - lse;
+      const double lpv = nucleus_lp(&nt[j], load_x(trow[j], a->dtype, v) / T - lse, v);
       if (dist) dist[v] = exp(lpv);
       const double score = lpv + (double)gj[v];
       if (score > best1) {
@@ -293,7 +361,7 @@ done:
     a->accept_len[b] = -1;
   }
   free(lse_t); free(lse_d); free(lqz); free(lp); free(logw); free(logpi);
-  free(s1); free(s2); free(lqv);
+  free(s1); free(s2); free(lqv); free(nt); free(nd);
   return flags;
 }
 
@@ -311,14 +379,15 @@ static void* verify_worker(void* p) {
 
 int oracle_verify(const void* target, const int32_t* target_row_off, const void* draft, int dtype,
                   const int32_t* tokens, const int32_t* verify_len, const float* u, const float* g,
-                  const float* mix_w, int K, int B, int L, int64_t V, double T, int n_threads,
+                  const float* mix_w, int K, int B, int L, int64_t V, double T, double top_p, int n_threads,
                   int32_t* accept_len, int32_t* out_tokens, const oracle_diag* diag) {
   if (!target || !draft || !tokens || !u || !g || !accept_len || !out_tokens) return ORC_ERR_ARG;
   if (dtype != ORC_F32 && dtype != ORC_BF16) return ORC_ERR_ARG;
   if (B < 0 || L < 0 || L > 64 || V < 1 || K < 1 || !(T > 0.0)) return ORC_ERR_ARG;
+  if (!(top_p > 0.0 && top_p <= 1.0)) return ORC_ERR_ARG;
   if (!mix_w && K != 1) return ORC_ERR_ARG;
   verify_args a = {target, target_row_off, draft, dtype, tokens, verify_len, u, g, mix_w,
-                   K, B, L, V, T, accept_len, out_tokens, diag};
+                   K, B, L, V, T, top_p, accept_len, out_tokens, diag};
   if (n_threads < 1) n_threads = 1;
   if (n_threads > B) n_threads = B > 0 ? B : 1;
   verify_job* jobs = calloc((size_t)n_threads, sizeof(verify_job));

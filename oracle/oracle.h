@@ -74,11 +74,16 @@ int oracle_softmax_T(const void* x, int dtype, int64_t rows, int64_t V, int64_t 
  *  tokens:  [B, L] drafted tokens x_i; u: [B, L] uniforms in [0, 1);
  *  g:       [B, L+1, V] Gumbel noise, indexed by (request, terminal position).
  *  verify_len: [B] (nullable -> L) number of positions that are tested.
+ *  top_p:   in (0, 1]; below 1 every row's temperature softmax is filtered to
+ *           its nucleus before use (the smallest set of most probable tokens,
+ *           ties to the lower index, whose mass reaches top_p, renormalised;
+ *           other tokens get probability 0), for the target and for every
+ *           draft category alike. 1 leaves the rows unfiltered.
  *  Outputs: accept_len [B], out_tokens [B, L+1] (accepted prefix, the
  *  terminal token, then -1). Returns ORC_ERR_ARG, or the OR of per-request flags. */
 int oracle_verify(const void* target, const int32_t* target_row_off, const void* draft, int dtype,
                   const int32_t* tokens, const int32_t* verify_len, const float* u, const float* g,
-                  const float* mix_w, int K, int B, int L, int64_t V, double T, int n_threads,
+                  const float* mix_w, int K, int B, int L, int64_t V, double T, double top_p, int n_threads,
                   int32_t* accept_len, int32_t* out_tokens, const oracle_diag* diag);
 
 /* DVL allocation: prefix-survival products P[b,i] = s[b,0]*...*s[b,i] (fp64,
