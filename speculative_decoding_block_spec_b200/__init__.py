@@ -9,10 +9,14 @@ is not on a CUDA device, the call raises.
 
 Entry points (same names as the C ABI):
   softmax_T(logits, T, probs=False)             temperature softmax statistics
+  spec_softmax_T(logits, T, row_max, row_lse, probs=None, workspace=None)
+  spec_softmax_T_noalloc(logits, T, row_max, row_lse, probs=None)
   spec_verify_block(target, draft, tokens, u, g, T, ...)
   spec_verify_mixture(target, draft, mix_w, tokens, u, g, T, ...)
+  spec_verify_window_stats(...), spec_verify_accept(...)   the two verify stages
   dvl_allocate_pack(scores, budget, dense_target=None, packed_target=None)
-Workspaces: Workspace(nbytes, device), with verify/softmax/dvl size helpers.
+Workspaces: Workspace(nbytes, device), with verify/softmax/dvl size helpers;
+Workspace.status() reads the sticky device flags (DEV_*).
 """
 import ctypes
 import os
