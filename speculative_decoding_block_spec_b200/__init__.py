@@ -25,7 +25,7 @@ import torch
 
 __all__ = ["SpecError", "Workspace", "lib", "softmax_T", "spec_softmax_T", "spec_softmax_T_noalloc", "NOALLOC_MAX_ROWS", "spec_verify_block",
            "spec_verify_mixture", "spec_verify_window_stats", "spec_verify_accept", "dvl_allocate_pack", "verify_workspace_size", "softmax_workspace_size",
-           "dvl_workspace_size", "LIB_PATH", "EXPORTS", "DEV_TOKEN_RANGE", "DEV_NONFINITE", "DEV_VERIFY_LEN",
+           "dvl_workspace_size", "check_verify_args", "LIB_PATH", "EXPORTS", "DEV_TOKEN_RANGE", "DEV_NONFINITE", "DEV_VERIFY_LEN",
            "DEV_SCORES"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libspecv.so")
@@ -146,9 +146,19 @@ def _opt(t, name, dtype):
     return None if t is None else _dev(t, name, dtype)
 
 
+def _softmax_shapes(logits, row_max, row_lse, probs):
+    _shape(logits, "logits", (None, None))
+    rows, V = logits.shape
+    _shape(row_max, "row_max", (rows,))
+    _shape(row_lse, "row_lse", (rows,))
+    if probs is not None:
+        _shape(probs, "probs", (rows, V))
+    return rows, V
+
+
 def spec_softmax_T(logits, T, row_max, row_lse, probs=None, workspace=None):
     """C-ABI spec_softmax_T on preallocated outputs. logits [rows, V] (row stride V)."""
-    rows, V = logits.shape
+    rows, V = _softmax_shapes(logits, row_max, row_lse, probs)
     ws = workspace or Workspace(softmax_workspace_size(rows), logits.device)
     _call("spec_softmax_T", _dev(logits, "logits"), _dtype_code(logits), rows, V, V, float(T),
           _dev(row_max, "row_max", torch.float32), _dev(row_lse, "row_lse", torch.float32),
@@ -160,7 +170,7 @@ def spec_softmax_T_noalloc(logits, T, row_max, row_lse, probs=None):
     """C-ABI spec_softmax_T_noalloc on preallocated outputs: spec_softmax_T with
     the library's fixed scratch instead of a workspace (rows <= NOALLOC_MAX_ROWS;
     calls on one device must not overlap on the GPU)."""
-    rows, V = logits.shape
+    rows, V = _softmax_shapes(logits, row_max, row_lse, probs)
     if rows > NOALLOC_MAX_ROWS:
         raise ValueError("spec_softmax_T_noalloc: %d rows exceed the fixed scratch limit of %d rows"
                          % (rows, NOALLOC_MAX_ROWS))
@@ -180,6 +190,56 @@ def softmax_T(logits, T, probs=False, workspace=None):
     return (rmax, rlse, p) if probs else (rmax, rlse)
 
 
+def _shape(t, name, shape):
+    """Raises unless tensor t has exactly `shape` (entries of None match any size)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a tensor" % name)
+    if t.dim() != len(shape) or any(want is not None and got != want for got, want in zip(t.shape, shape)):
+        raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape),
+                                                            tuple("*" if w is None else w for w in shape)))
+
+
+def check_verify_args(target, draft, tokens, u, g, *, mix_w=None, verify_len=None, target_row_off=None,
+                      out=None, mixture=None):
+    """Host-side shape and device checks of a verify call, done before any
+    pointer reaches the library (the C ABI sees raw pointers and cannot tell a
+    short tensor from a long one). Returns (B, L, K, V). mixture=None infers
+    the draft layout from its rank: [B, L, V] (K = 1) or [B, K, L, V]."""
+    _shape(tokens, "tokens", (None, None))
+    B, L = tokens.shape
+    if mixture is None:
+        mixture = draft.dim() == 4
+    if mixture:
+        _shape(draft, "draft", (B, None, L, None))
+        K = draft.shape[1]
+    else:
+        _shape(draft, "draft", (B, L, None))
+        K = 1
+    V = draft.shape[-1]
+    if target_row_off is None:
+        _shape(target, "target", (B, L + 1, V))
+    else:
+        _shape(target, "target", (None, V))
+        if target.shape[0] < L + 1:
+            raise ValueError("packed target has %d rows, fewer than one request's L+1 = %d" % (target.shape[0], L + 1))
+        if target_row_off.dim() != 1 or target_row_off.numel() < B:
+            raise ValueError("target_row_off must be 1-D with at least B = %d entries" % B)
+    _shape(u, "u", (B, L))
+    _shape(g, "g", (B, L + 1, V))
+    if mix_w is not None:
+        _shape(mix_w, "mix_w", (B, K))
+    if verify_len is not None and (verify_len.dim() != 1 or verify_len.numel() < B):
+        raise ValueError("verify_len must be 1-D with at least B = %d entries" % B)
+    if out is not None:
+        _shape(out[0], "accept_len", (B,))
+        _shape(out[1], "out_tokens", (B, L + 1))
+    tensors = [target, draft, tokens, u, g, mix_w, verify_len, target_row_off] + list(out or [])
+    devs = {t.device for t in tensors if t is not None}
+    if len(devs) > 1:
+        raise ValueError("all tensors of a verify call must be on one device, got %s" % sorted(map(str, devs)))
+    return B, L, K, V
+
+
 def _outputs(B, L, device, out):
     if out is None:
         return (torch.empty(B, dtype=torch.int32, device=device),
@@ -192,8 +252,8 @@ def spec_verify_block(target, draft, tokens, u, g, T, *, verify_len=None, target
     """Verify B independently drafted blocks. target [B, L+1, V] (or packed rows
     [S, V] with target_row_off [B]), draft [B, L, V], tokens [B, L] int32,
     u [B, L] fp32, g [B, L+1, V] fp32. Returns (accept_len [B], out_tokens [B, L+1])."""
-    B, L = tokens.shape
-    V = draft.shape[-1]
+    B, L, _, V = check_verify_args(target, draft, tokens, u, g, verify_len=verify_len,
+                                   target_row_off=target_row_off, out=out, mixture=False)
     ws = workspace or Workspace(verify_workspace_size(B, L, 1, V), draft.device)
     acc, outt = _outputs(B, L, draft.device, out)
     if _dtype_code(target) != _dtype_code(draft):
@@ -210,8 +270,8 @@ def spec_verify_mixture(target, draft, mix_w, tokens, u, g, T, *, verify_len=Non
                         workspace=None, out=None):
     """Verify B latent-mixture drafts: draft [B, K, L, V], mix_w [B, K] fp32
     (category probabilities q(z|y)); other arguments as spec_verify_block."""
-    B, L = tokens.shape
-    K, V = draft.shape[1], draft.shape[-1]
+    B, L, K, V = check_verify_args(target, draft, tokens, u, g, mix_w=mix_w, verify_len=verify_len,
+                                   target_row_off=target_row_off, out=out, mixture=True)
     ws = workspace or Workspace(verify_workspace_size(B, L, K, V), draft.device)
     acc, outt = _outputs(B, L, draft.device, out)
     if _dtype_code(target) != _dtype_code(draft):
@@ -229,9 +289,15 @@ def spec_verify_window_stats(target, draft, tokens, T, workspace, *, verify_len=
     """Stage 1 of verification: temperature-softmax statistics of the verify
     window, and each row's logit at the drafted token, into `workspace`
     (draft [B, L, V] for K == 1, else [B, K, L, V]; tokens [B, L] int32)."""
+    _shape(tokens, "tokens", (None, None))
     B, L = tokens.shape
+    _shape(draft, "draft", (B, L, None) if draft.dim() == 3 else (B, None, L, None))
     K = 1 if draft.dim() == 3 else draft.shape[1]
     V = draft.shape[-1]
+    if target_row_off is None:
+        _shape(target, "target", (B, L + 1, V))
+    else:
+        _shape(target, "target", (None, V))
     _call("spec_verify_window_stats", _dev(target, "target"), _opt(target_row_off, "target_row_off", torch.int32),
           _dev(draft, "draft"), K, _dtype_code(draft), _dev(tokens, "tokens", torch.int32),
           _opt(verify_len, "verify_len", torch.int32), B, L, V, float(T), workspace.ptr(), workspace.nbytes,
@@ -242,9 +308,8 @@ def spec_verify_accept(target, draft, tokens, u, g, T, workspace, *, mix_w=None,
                        target_row_off=None, out=None):
     """Stage 2 of verification (after spec_verify_window_stats on the same
     workspace): accept tests, first rejection and the terminal draw."""
-    B, L = tokens.shape
-    K = 1 if draft.dim() == 3 else draft.shape[1]
-    V = draft.shape[-1]
+    B, L, K, V = check_verify_args(target, draft, tokens, u, g, mix_w=mix_w, verify_len=verify_len,
+                                   target_row_off=target_row_off, out=out)
     acc, outt = _outputs(B, L, draft.device, out)
     _call("spec_verify_accept", _dev(target, "target"), _opt(target_row_off, "target_row_off", torch.int32),
           _dev(draft, "draft"), _opt(mix_w, "mix_w", torch.float32), K, _dtype_code(draft),
@@ -260,8 +325,20 @@ def dvl_allocate_pack(scores, budget, *, dense_target=None, packed_target=None, 
     Returns (verify_len [B], offsets [B+1], slot_map [budget]) int32; if
     dense_target [B, L+1, V] and packed_target [budget, V] are given, the
     selected rows are copied into packed_target."""
+    _shape(scores, "scores", (None, None))
     B, L = scores.shape
     dev = scores.device
+    if out is not None:
+        _shape(out[0], "verify_len", (B,))
+        _shape(out[1], "offsets", (B + 1,))
+        if out[2] is not None and (out[2].dim() != 1 or out[2].numel() < int(budget)):
+            raise ValueError("slot_map must be 1-D with at least budget = %d entries" % int(budget))
+    if dense_target is not None:
+        _shape(dense_target, "dense_target", (B, L + 1, None))
+    if packed_target is not None:
+        _shape(packed_target, "packed_target", (None, None if dense_target is None else dense_target.shape[-1]))
+        if packed_target.shape[0] < int(budget):
+            raise ValueError("packed_target has %d rows, fewer than budget = %d" % (packed_target.shape[0], int(budget)))
     ws = workspace or Workspace(dvl_workspace_size(B), dev)
     if out is None:
         out = (torch.empty(B, dtype=torch.int32, device=dev), torch.empty(B + 1, dtype=torch.int32, device=dev),
