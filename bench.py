@@ -301,6 +301,7 @@ def main():
     import torch.distributed as dist
     import speculative_decoding_block_spec_b200 as specv
     from speculative_decoding_block_spec_b200 import synth
+    from speculative_decoding_block_spec_b200.dist import max_over_ranks as _max_over_ranks
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -385,11 +386,8 @@ def main():
         torch.cuda.synchronize(dev)
 
     def max_over_ranks(ms):
-        if world == 1:
-            return ms
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        """The slowest rank's time (the value itself on one GPU)."""
+        return _max_over_ranks(ms, dev)
 
     sampler = ClockSampler(local)
     wall = {}
