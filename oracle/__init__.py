@@ -36,7 +36,7 @@ def _load():
 class _Diag(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "lp", "lq", "rho", "accept_margin", "terminal_row", "terminal_kind",
-        "argmax_gap", "argmax_kappa", "terminal_dist")]
+        "argmax_gap", "argmax_kappa", "terminal_dist", "nucleus_margin")]
 
 
 def _ptr(a):
@@ -102,7 +102,7 @@ def verify(target, draft, tokens, u, g, T, *, mix_w=None, verify_len=None, targe
         res = dict(lp=np.empty((B, L)), lq=np.empty((B, L)), rho=np.empty((B, L)),
                    accept_margin=np.empty((B, L)), terminal_row=np.empty(B, np.int32),
                    terminal_kind=np.empty(B, np.int32), argmax_gap=np.empty(B),
-                   argmax_kappa=np.empty(B), terminal_dist=np.empty((B, V)))
+                   argmax_kappa=np.empty(B), terminal_dist=np.empty((B, V)), nucleus_margin=np.empty(B))
         dptr = ctypes.byref(_Diag(*[_ptr(res[f[0]]) for f in _Diag._fields_]))
     st = _load().oracle_verify(_ptr(target), _ptr(off), _ptr(draft), dt, _ptr(tokens), _ptr(vl),
                                _ptr(u), _ptr(g), _ptr(w), K, B, L, V, float(T), float(top_p), int(n_threads),

@@ -97,6 +97,7 @@ typedef struct {
   double lp_cut;    /* log-probability of the last member */
   int64_t v_cut;    /* its token; equal log-probabilities are members up to it */
   double log_mass;  /* log of the nucleus mass */
+  double margin;    /* min(mass with the last member - top_p, top_p - mass without it) */
 } nucleus;
 
 typedef struct { double lp; int64_t v; } ranked;
@@ -114,6 +115,7 @@ static void row_nucleus(const void* row, int dtype, int64_t V, double T, double 
   n->lp_cut = -INFINITY;
   n->v_cut = V - 1;
   n->log_mass = 0.0;
+  n->margin = INFINITY;
   if (n->all) return;
   ranked* r = malloc((size_t)V * sizeof(ranked));
   for (int64_t v = 0; v < V; ++v) {
@@ -121,13 +123,19 @@ static void row_nucleus(const void* row, int dtype, int64_t V, double T, double 
     r[v].v = v;
   }
   qsort(r, (size_t)V, sizeof(ranked), ranked_order);
-  double mass = 0.0;
+  double mass = 0.0, before = 0.0;
   int64_t k = 0;
   for (; k < V; ++k) {
+    before = mass;
     mass += exp(r[k].lp);
     if (mass >= top_p) break;
   }
-  if (k == V) k = V - 1; /* rounding kept the total just below top_p: the whole row */
+  if (k == V) { /* rounding kept the total just below top_p: the whole row */
+    k = V - 1;
+    n->margin = top_p - mass;
+  } else {
+    n->margin = fmin(mass - top_p, top_p - before);
+  }
   n->lp_cut = r[k].lp;
   n->v_cut = r[k].v;
   n->log_mass = log(mass);
@@ -207,6 +215,7 @@ static int verify_one(const verify_args* a, int b) {
     if (d->argmax_kappa) d->argmax_kappa[b] = NAN;
     if (d->terminal_dist)
       for (int64_t v = 0; v < V; ++v) d->terminal_dist[(int64_t)b * V + v] = 0.0;
+    if (d->nucleus_margin) d->nucleus_margin[b] = NAN;
   }
 
   const int ell = a->verify_len ? a->verify_len[b] : L;
@@ -345,6 +354,16 @@ static int verify_one(const verify_args* a, int b) {
   out[j] = (int32_t)t;
   a->accept_len[b] = j;
   if (d) {
+    if (d->nucleus_margin) { /* rows 0..j of target and drafts (their tests and the residual), or the bonus row */
+      double mg = INFINITY;
+      const int last = j < ell ? j : ell - 1;
+      for (int i = 0; i <= last; ++i) {
+        mg = fmin(mg, nt[i].margin);
+        for (int z = 0; z < K; ++z) mg = fmin(mg, nd[z * L + i].margin);
+      }
+      if (j == ell) mg = fmin(mg, nt[ell].margin);
+      d->nucleus_margin[b] = mg;
+    }
     if (d->terminal_row) d->terminal_row[b] = j;
     if (d->terminal_kind) d->terminal_kind[b] = kind;
     if (d->argmax_gap) d->argmax_gap[b] = best1 - best2; /* +inf with a single candidate */

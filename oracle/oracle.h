@@ -58,6 +58,9 @@ typedef struct {
   double* argmax_gap;    /* [B] fp64 gap between the two best terminal scores (+inf if one candidate) */
   double* argmax_kappa;  /* [B] max(1, kappa of the two best); kappa_v = p_v / (p_v - q_v) */
   double* terminal_dist; /* [B*V] normalised distribution the terminal token is a Gumbel-max draw from */
+  double* nucleus_margin;/* [B] top_p < 1: smallest distance between top_p and the cumulative masses on
+                            either side of the nucleus cut, over the rows the outputs depend on (+inf
+                            for top_p = 1): below 1e-6 the nucleus itself is a low-margin decision */
 } oracle_diag;
 
 /* Temperature softmax of each row: z = x / T, row_max = max z,

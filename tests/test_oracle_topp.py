@@ -202,6 +202,31 @@ def test_exact_enumeration_is_lossless_under_the_filter(K, top_p):
             np.testing.assert_allclose(mass, pf[k] * mass.sum(), rtol=0, atol=1e-13)
 
 
+@pytest.mark.parametrize("top_p,expect", [(0.4, 0.1), (0.6, 0.1), (0.75, 0.05), (0.9, 0.1), (1.0, np.inf)])
+def test_nucleus_margin_is_the_distance_to_the_cut(top_p, expect):
+    """p = (0.5, 0.3, 0.2): the cumulative masses are 0.5, 0.8 and 1, and the
+    margin is the distance from top_p to the masses just before and at the
+    cut (e.g. 0.75 -> min(0.8 - 0.75, 0.75 - 0.5) = 0.05)."""
+    row = np.log(np.array([0.5, 0.3, 0.2])).astype(np.float32)  # fp32 logits: p within ~1e-7 of these
+    target = np.broadcast_to(row, (1, 2, 3)).copy()
+    r = oracle.verify(target, target[:, :1].copy(), np.zeros((1, 1), np.int32), np.zeros((1, 1), np.float32),
+                      np.zeros((1, 2, 3), np.float32), 1.0, verify_len=np.zeros(1, np.int32), diag=True,
+                      top_p=top_p)
+    m = r["nucleus_margin"][0]
+    assert np.isinf(m) if np.isinf(expect) else abs(m - expect) < 1e-6
+
+
+def test_nucleus_margin_takes_the_smallest_over_the_rows_used():
+    """Target row 0 (0.5, 0.3, 0.2) has margin 0.05 at top_p 0.75; draft row 0
+    (0.74, 0.16, 0.1) has min(0.9 - 0.75, 0.75 - 0.74) = 0.01, the request's."""
+    t = np.log(np.array([[0.5, 0.3, 0.2], [0.5, 0.3, 0.2]])).astype(np.float32)[None]
+    d = np.log(np.array([[0.74, 0.16, 0.1]])).astype(np.float32)[None]
+    for uu in (0.0, 0.999):  # accepted (bonus row used) or rejected (residual on row 0)
+        r = oracle.verify(t, d, np.zeros((1, 1), np.int32), np.full((1, 1), uu, np.float32),
+                          np.zeros((1, 2, 3), np.float32), 1.0, diag=True, top_p=0.75)
+        assert r["flags"] == 0 and abs(r["nucleus_margin"][0] - 0.01) < 1e-6
+
+
 def test_rejects_bad_top_p():
     x = np.zeros((1, 2, 4), np.float32)
     for bad in (0.0, -0.5, 1.5, float("nan")):
