@@ -1,25 +1,35 @@
 #!/usr/bin/env python
 """Benchmark of batched speculative-draft verification on B200.
 
-One step = one pass of the whole hot path over one batch: the fused
-temperature-softmax statistics of the verify window, the accept tests with
-first-rejection ballot, and the residual / bonus Gumbel-max draw (plus DVL
-allocation and packing for the DVL workloads). Metric: verified
+One step = one pass of the whole hot path over one batch: DVL allocation
+(for the workloads with a verify budget), the fused temperature-softmax
+statistics of the verify window, the accept tests with first-rejection
+ballot, and the residual / bonus Gumbel-max draw. Metric: verified
 request-blocks per second (one request-block = one request's verify step),
 with the achieved HBM bandwidth against the measured B200 copy peak.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2] [--impl specv|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 5] [--extras 2,3,4]
+                    [--impl specv|reference]
+
+The headline workload is the stress case (B=64, L=16, V=151936, K=4
+latent-mixture drafts, bf16, DVL budget 544 = half of B(L+1)), the largest
+of the five seeded workloads; --extras measures further workloads in the
+same run with the same protocol and reports them under "workloads".
 
 Under torchrun every rank verifies its own batch (weak scaling, no
 collective on the data path); the time is the max over ranks. Prints one
 JSON line on rank 0.
 
-Timing: inputs live in HBM; 4 rotating input sets (each > 160 MB, together
-far above the 126 MB L2) so each step reads its logits from HBM; each step is
-a CUDA-graph replay of the library's launches; CUDA events on the launching
-stream. The dominant kernel (row statistics) is also timed alone with
-events to give the roofline fraction. The e2e leg copies each step's inputs
-from pinned host memory and reads the results back inside the timed region.
+Timing: inputs live in HBM; --sets rotating input sets (4 by default, each
+above 160 MB, together far above the 126 MB L2), so each step reads its
+logits from HBM. The headline `value` is K CUDA-graph replays of the step
+between one pair of CUDA events on the launching stream. The same step is
+also timed replay by replay (one event pair each; median and spread), both
+as graph replays and as plain stream launches through the public API, which
+gives the launch-gap saving of the captured graph. The dominant kernel (row
+statistics) is timed alone with events for the roofline fraction. The e2e
+leg copies each step's inputs from pinned host memory and reads the results
+back inside the timed region.
 """
 import argparse
 import glob
@@ -29,7 +39,6 @@ import os
 import re
 import statistics
 import sys
-import threading
 import time
 
 import numpy as np
@@ -40,20 +49,28 @@ sys.path.insert(0, ROOT)
 METRIC = "verified request-blocks/sec and achieved HBM GB/s (% of B200 peak), 1 GPU"
 UNIT = "request-blocks/s"
 NOMINAL_HBM_GBS = 8000.0
-NSETS = 4
+L2_BYTES = 126 * 2 ** 20
+HEADLINE = 5
+EPS_MARGIN = 1e-6
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5000)
-    ap.add_argument("--warmup", type=int, default=100)
-    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--workload", type=int, default=HEADLINE, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--extras", default="2,3,4",
+                    help="comma-separated further workloads measured in the same run ('' for none)")
+    ap.add_argument("--sets", type=int, default=4, help="rotating input sets (together above the L2 size)")
     ap.add_argument("--impl", default="specv", choices=["specv", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU-baseline sample")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    return ap.parse_args()
+    args = ap.parse_args(argv)
+    args.extra_ids = [int(c) for c in args.extras.split(",") if c.strip()] if args.extras else []
+    args.extra_ids = [c for c in args.extra_ids if c != args.workload]
+    return args
 
 
 def measured_peaks():
@@ -62,7 +79,7 @@ def measured_peaks():
             p = json.load(f)
         return float(p["hbm_gbs"]), "MEASURED_PEAKS.json hbm_gbs (1 Gi bf16 copy, burst) of measured"
     except (OSError, KeyError, ValueError):
-        return 6650.0, "fallback 6.65 TB/s"
+        return 6650.0, "fallback 6.65 TB/s (MEASURED_PEAKS.json absent)"
 
 
 # ---------------------------------------------------------------- workload
@@ -76,8 +93,13 @@ def window_bytes(w, verify_len):
 
 def step_bytes(w, verify_len, accept_len):
     """Algorithmic bytes of one verify step: the window, one fp32 Gumbel row
-    per request, the bonus target row of requests that accepted every tested
-    position, and the small per-request arrays."""
+    per request, the bonus target row of the requests that accepted every
+    tested position, and the small per-request arrays.
+
+    The bonus row is counted only where the method reads it (a request that
+    accepted all of its l_b positions draws its last token from target row
+    l_b); the survey's byte model counts (l_b + 1) target rows for every
+    request, which overstates the bytes of requests that reject."""
     e = 2 if w.dtype == "bf16" else 4
     bonus = sum(1 for l, a in zip(verify_len, accept_len) if a == l)
     small = w.B * (w.L * 4 * 2 + 4 + (w.L + 1) * 4)
@@ -86,12 +108,42 @@ def step_bytes(w, verify_len, accept_len):
     return window_bytes(w, verify_len) + w.B * w.V * 4 + bonus * w.V * e + small
 
 
+def set_bytes(w):
+    """Device bytes of one input set: target (dense, plus the packed rows with
+    a budget), draft, Gumbel noise and the small arrays."""
+    e = 2 if w.dtype == "bf16" else 4
+    n = w.B * (w.L + 1) * w.V * e + w.B * w.K * w.L * w.V * e + w.B * (w.L + 1) * w.V * 4
+    n += w.B * w.L * 8 + (w.B * w.K * 4 if w.K > 1 else 0)
+    if w.budget is not None:
+        n += w.budget * w.V * e + w.B * w.L * 4
+    return n
+
+
+def l2_note(w, nsets):
+    return "%d rotating input sets of %.0f MB (%s the 126 MB L2 together)" % (
+        nsets, set_bytes(w) / 1e6, "above" if nsets * set_bytes(w) > L2_BYTES else "NOT above")
+
+
+def config_of(w, nsets, world):
+    """The workload description shared by both arms (same keys and values)."""
+    return {"workload": w.name, "B": w.B, "L": w.L, "V": w.V, "K": w.K, "T": w.T, "budget": w.budget,
+            "l2": l2_note(w, nsets), "parallelism": "dp%d" % world}
+
+
+def spread(ms):
+    """Median and spread of per-replay times (ms)."""
+    a = np.sort(np.asarray(ms, np.float64))
+    q = lambda f: float(a[min(len(a) - 1, int(round(f * (len(a) - 1))))])
+    return {"median_ms": q(0.5), "p10_ms": q(0.1), "p90_ms": q(0.9), "min_ms": float(a[0]), "max_ms": float(a[-1]),
+            "n": int(len(a))}
+
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
     """nvidia-smi in its own process (`-lms`), started before the warm-up and
     stopped after the timed region; the report keeps the samples whose
-    timestamps fall inside the timed region."""
+    timestamps fall inside the timed region. It only reads the clocks."""
 
     FIELDS = ["timestamp", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
               "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
@@ -103,7 +155,9 @@ class ClockSampler:
         self.region = None
         self.err = None
         self.proc = None
-        self.path = tempfile.mktemp(prefix="clocks_", suffix=".csv")
+        self.period_ms = period_ms
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
         try:
             import torch
             uuid = str(torch.cuda.get_device_properties(cuda_index).uuid)
@@ -148,10 +202,11 @@ class ClockSampler:
             return {"error": "no nvidia-smi samples"}
         t0, t1 = self.region
         inside = [r for r in rows if t0 <= r[0] <= t1]
-        note = "nvidia-smi -lms 20 during the timed region"
+        note = "nvidia-smi -lms %d during the timed region" % self.period_ms
         if not inside:
             inside = sorted(rows, key=lambda r: min(abs(r[0] - t0), abs(r[0] - t1)))[:2]
-            note = "nvidia-smi -lms 20, the samples nearest the timed region (region shorter than the period)"
+            note = "nvidia-smi -lms %d, the samples nearest the timed region (region shorter than the period)" \
+                   % self.period_ms
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         active = sorted({names[k] for r in inside for k, v in enumerate(r[3]) if v.lower().startswith("active")})
         return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": inside[0][2], "reasons": active,
@@ -160,23 +215,67 @@ class ClockSampler:
 
 # ------------------------------------------------------------ the oracle leg
 
-def oracle_sample(x, requests, n_threads):
-    """One oracle verify over the first `requests` requests of inputs x."""
+def oracle_sample(x, requests, n_threads, diag=False):
+    """One oracle verify over the first `requests` requests of inputs x (with
+    a budget: the oracle's own allocation and packing of the whole batch)."""
     import oracle
     w = x.w
     sl = slice(0, requests)
     if w.budget is None:
         return oracle.verify(x.target[sl], x.draft[sl], x.tokens[sl], x.u[sl], x.g[sl], w.T,
-                             mix_w=None if x.mix_w is None else x.mix_w[sl], n_threads=n_threads)
+                             mix_w=None if x.mix_w is None else x.mix_w[sl], n_threads=n_threads, diag=diag)
     rd = oracle.dvl_allocate(x.scores, w.budget)
     packed = oracle.pack(x.target, rd["verify_len"], rd["offsets"], w.budget)
-    return oracle.verify(packed, x.draft[sl], x.tokens[sl], x.u[sl], x.g[sl], w.T,
-                         mix_w=None if x.mix_w is None else x.mix_w[sl], verify_len=rd["verify_len"][sl],
-                         target_row_off=rd["offsets"][:w.B][sl], n_threads=n_threads)
+    r = oracle.verify(packed, x.draft[sl], x.tokens[sl], x.u[sl], x.g[sl], w.T,
+                      mix_w=None if x.mix_w is None else x.mix_w[sl], verify_len=rd["verify_len"][sl],
+                      target_row_off=rd["offsets"][:w.B][sl], n_threads=n_threads, diag=diag)
+    r["verify_len"] = rd["verify_len"][sl]
+    return r
 
 
-def cpu_baseline(x, seconds):
-    """The oracle as it stands, on this host's cores, repeated for about `seconds`."""
+def margin_report(acc, out, ref, verify_len):
+    """Decisions of one verify call and the low-margin ones among them, as the
+    parity rule counts them: every tested accept decision and the terminal
+    draw; an accept test is low-margin when |u - min(1, rho)| < 1e-6, a draw
+    when the fp64 gap between its two best scores is below 1e-6 * max(1,
+    kappa). `mismatches` counts GPU outputs that differ from the oracle's
+    outside the low-margin exemption (0 is parity)."""
+    n_dec = n_low = n_exempt_diff = n_bad = 0
+    L = out.shape[1] - 1
+    for b in range(out.shape[0]):
+        ja = int(ref["accept_len"][b])
+        if ja < 0:
+            n_bad += int(not (acc[b] == -1 and np.all(out[b] == -1)))
+            continue
+        ell = L if verify_len is None else int(verify_len[b])
+        tested = ja + 1 if ja < ell else ja
+        m = ref["accept_margin"][b]
+        n_dec += tested + 1
+        low = [i for i in range(tested) if m[i] < EPS_MARGIN]
+        same = acc[b] == ja and np.array_equal(out[b], ref["out_tokens"][b])
+        if low:  # exempt from the first low-margin test on; the outputs before it must still match
+            n_low += 1
+            i0 = low[0]
+            before_ok = acc[b] >= i0 and np.array_equal(out[b, :i0], ref["out_tokens"][b][:i0])
+            n_bad += int(not same and not before_ok)
+            n_exempt_diff += int(not same and before_ok)
+            continue
+        if ref["argmax_gap"][b] < EPS_MARGIN * max(1.0, ref["argmax_kappa"][b]):
+            n_low += 1
+            same_prefix = acc[b] == ja and np.array_equal(out[b, :ja], ref["out_tokens"][b, :ja])
+            n_bad += int(not same_prefix)
+            n_exempt_diff += int(same_prefix and not same)
+            continue
+        n_bad += int(not same)
+    return {"decisions": n_dec, "low_margin": n_low, "low_margin_fraction": n_low / max(1, n_dec),
+            "exempted_differences": n_exempt_diff, "mismatches": n_bad}
+
+
+def cpu_baseline(x, seconds, gpu_out=None):
+    """The oracle as it stands, on this host's cores, repeated for about
+    `seconds`. With the GPU's outputs on the same inputs, one further oracle
+    run with diagnostics (outside the timed loop) counts the decisions and
+    the low-margin ones, and checks the GPU's outputs against it."""
     import oracle
     cores = oracle.n_cores()
     w = x.w
@@ -188,9 +287,15 @@ def cpu_baseline(x, seconds):
         if time.perf_counter() - t0 >= seconds:
             break
     dt = time.perf_counter() - t0
-    return {"value": reps * w.B / dt, "unit": UNIT, "cores": min(cores, w.B), "kind": "oracle",
-            "sample": "full workload (%d requests) x %d repetitions, %.1f s; fp64 C oracle, pthreads over requests"
-                      % (w.B, reps, dt)}
+    res = {"value": reps * w.B / dt, "unit": UNIT, "cores": min(cores, w.B), "kind": "oracle",
+           "sample": "full workload (%d requests) x %d repetitions, %.1f s; fp64 C oracle, pthreads over requests"
+                     % (w.B, reps, dt)}
+    margins = None
+    if gpu_out is not None:
+        ref = oracle_sample(x, w.B, cores, diag=True)
+        margins = margin_report(gpu_out[0], gpu_out[1], ref, ref.get("verify_len"))
+        margins["source"] = "oracle with diagnostics on input set 0, against the GPU's outputs on it"
+    return res, margins
 
 
 def run_reference(args, rank, world):
@@ -236,8 +341,7 @@ def run_reference(args, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic (seeded)", "config": {"workload": w.name, "B": w.B, "L": w.L, "V": w.V, "K": w.K,
-                                                     "T": w.T, "budget": w.budget},
+            "data": "synthetic (seeded)", "config": config_of(w, args.sets, world),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(cores, req), "kind": "oracle",
                              "sample": sample + " (%s); fp64 C oracle on the host cores" % w.name},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -251,7 +355,8 @@ def stats_kernel_name(w, sms):
     """The statistics kernel the library picks for this workload: the
     one-block-per-SM balanced kernel for 16-byte rows, windows of at most
     256 MB, at least 4096 units (2 KB slices for 32 warps) per SM and at most
-    32 rows per SM share; otherwise the even-split kernel."""
+    32 rows per SM share; otherwise the even-split kernel. The window bound
+    is the dense one, B (K+1) L rows."""
     esz = 2 if w.dtype == "bf16" else 4
     if (w.V * esz) % 16:
         return "k_row_stats"
@@ -261,7 +366,6 @@ def stats_kernel_name(w, sms):
     if units * 16 <= (256 << 20) and share >= 32 * 128 and -(-share // vu) + 1 <= 32:
         return "k_row_stats_dyn"
     return "k_row_stats"
-
 
 
 def committed_traffic(kernel, workload_name):
@@ -287,69 +391,56 @@ def committed_traffic(kernel, workload_name):
 
 # -------------------------------------------------------------- specv leg
 
-def main():
-    args = parse_args()
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.warmup < 3:
-        raise SystemExit("--warmup must be >= 3")
-    if args.impl == "reference":
-        return run_reference(args, rank, world)
+class Runner:
+    """Device-side state of one workload: its rotating input sets, the step
+    through the public API, and the CUDA graphs that replay it."""
 
-    import torch
-    import torch.distributed as dist
-    import speculative_decoding_block_spec_b200 as specv
-    from speculative_decoding_block_spec_b200 import synth
-    from speculative_decoding_block_spec_b200.dist import max_over_ranks as _max_over_ranks
+    def __init__(self, w, x, dev, stream, nsets):
+        import torch
+        import speculative_decoding_block_spec_b200 as specv
+        self.torch, self.specv = torch, specv
+        self.w, self.x, self.dev, self.stream = w, x, dev, stream
 
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        def logits(a):
+            if a.dtype == np.uint16:
+                return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+            return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
 
-    w = synth.WORKLOADS[args.workload]
-    x = synth.make_inputs(w, seed=rank)  # weak scaling: every rank verifies its own batch
-    stream = torch.cuda.Stream(dev)
+        self.sets = []
+        with torch.cuda.stream(stream):
+            for _ in range(nsets):
+                d = dict(target=logits(x.target), draft=logits(x.draft), tokens=torch.from_numpy(x.tokens).to(dev),
+                         u=torch.from_numpy(x.u).to(dev), g=torch.from_numpy(x.g).to(dev))
+                if x.mix_w is not None:
+                    d["mix_w"] = torch.from_numpy(x.mix_w).to(dev)
+                if x.scores is not None:
+                    d["scores"] = torch.from_numpy(x.scores).to(dev)
+                    d["packed"] = torch.zeros((w.budget, w.V), dtype=d["target"].dtype, device=dev)
+                    d["dvl_ws"] = specv.Workspace(specv.dvl_workspace_size(w.B), dev)
+                    d["dvl_out"] = (torch.empty(w.B, dtype=torch.int32, device=dev),
+                                    torch.empty(w.B + 1, dtype=torch.int32, device=dev),
+                                    torch.empty(w.budget, dtype=torch.int32, device=dev))
+                d["ws"] = specv.Workspace(specv.verify_workspace_size(w.B, w.L, w.K, w.V), dev)
+                d["out"] = (torch.empty(w.B, dtype=torch.int32, device=dev),
+                            torch.empty((w.B, w.L + 1), dtype=torch.int32, device=dev))
+                self.sets.append(d)
+            stream.synchronize()
+        self.launches_per_step = (2 if w.L > 0 else 1) + (1 if w.budget is not None else 0)
+        self.graphs = {}
 
-    def logits(a):
-        if a.dtype == np.uint16:
-            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
-        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
-
-    sets = []
-    with torch.cuda.stream(stream):
-        for s in range(NSETS):
-            d = dict(target=logits(x.target), draft=logits(x.draft), tokens=torch.from_numpy(x.tokens).to(dev),
-                     u=torch.from_numpy(x.u).to(dev), g=torch.from_numpy(x.g).to(dev))
-            if x.mix_w is not None:
-                d["mix_w"] = torch.from_numpy(x.mix_w).to(dev)
-            if x.scores is not None:
-                d["scores"] = torch.from_numpy(x.scores).to(dev)
-                d["packed"] = torch.zeros((w.budget, w.V), dtype=d["target"].dtype, device=dev)
-                d["dvl_ws"] = specv.Workspace(specv.dvl_workspace_size(w.B), dev)
-                d["dvl_out"] = (torch.empty(w.B, dtype=torch.int32, device=dev),
-                                torch.empty(w.B + 1, dtype=torch.int32, device=dev),
-                                torch.empty(w.budget, dtype=torch.int32, device=dev))
-            d["ws"] = specv.Workspace(specv.verify_workspace_size(w.B, w.L, w.K, w.V), dev)
-            d["out"] = (torch.empty(w.B, dtype=torch.int32, device=dev),
-                        torch.empty((w.B, w.L + 1), dtype=torch.int32, device=dev))
-            sets.append(d)
-    set_bytes = sum(t.numel() * t.element_size() for k, t in sets[0].items() if isinstance(t, torch.Tensor))
-
-    def prepack(d):
+    def prepack(self, d):
         """DVL allocation plus the copy of the selected dense target rows into
         the fixed-address packed buffer. In deployment the target model writes
         its logits straight into the packed slots, so the copy is not part of
         the verify step: it runs once per input set here and is timed apart."""
-        specv.dvl_allocate_pack(d["scores"], w.budget, dense_target=d["target"], packed_target=d["packed"],
-                                workspace=d["dvl_ws"], out=d["dvl_out"])
+        self.specv.dvl_allocate_pack(d["scores"], self.w.budget, dense_target=d["target"],
+                                     packed_target=d["packed"], workspace=d["dvl_ws"], out=d["dvl_out"])
 
-    def step(d):
+    def step(self, d):
         """One verify step through the public API (the launches a user makes):
         with a DVL budget, the allocation over the survival scores, then
         verification of the packed rows at the allocated offsets."""
+        w, specv = self.w, self.specv
         vl = off = None
         target = d["target"]
         if w.budget is not None:
@@ -362,22 +453,72 @@ def main():
         return specv.spec_verify_mixture(target, d["draft"], d["mix_w"], d["tokens"], d["u"], d["g"], w.T,
                                          verify_len=vl, target_row_off=off, workspace=d["ws"], out=d["out"])
 
-    launches_per_step = (2 if w.L > 0 else 1) + (1 if w.budget is not None else 0)
+    def _window(self, d):
+        if self.w.budget is not None:
+            return d["dvl_out"][0], d["dvl_out"][1][:self.w.B], d["packed"]
+        return None, None, d["target"]
 
-    # capture one graph per input set; replay round-robin
-    graphs = []
-    with torch.cuda.stream(stream):
-        for d in sets:  # warm the occupancy cache and the kernels before capture
-            if w.budget is not None:
-                prepack(d)
-            step(d)
-        stream.synchronize()
-        for d in sets:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                step(d)
-            graphs.append(g)
-        stream.synchronize()
+    def verify_only(self, d):
+        """The verify call alone (the DVL outputs of the last step stay fixed)."""
+        w, specv = self.w, self.specv
+        vl, off, target = self._window(d)
+        if w.K == 1:
+            specv.spec_verify_block(target, d["draft"], d["tokens"], d["u"], d["g"], w.T, verify_len=vl,
+                                    target_row_off=off, workspace=d["ws"], out=d["out"])
+        else:
+            specv.spec_verify_mixture(target, d["draft"], d["mix_w"], d["tokens"], d["u"], d["g"], w.T,
+                                      verify_len=vl, target_row_off=off, workspace=d["ws"], out=d["out"])
+
+    def stats_only(self, d):
+        """Stage 1 alone: the statistics kernel, the dominant launch."""
+        vl, off, target = self._window(d)
+        self.specv.spec_verify_window_stats(target, d["draft"], d["tokens"], self.w.T, d["ws"], verify_len=vl,
+                                            target_row_off=off)
+
+    def capture(self, name, fn):
+        torch = self.torch
+        gs = []
+        with torch.cuda.stream(self.stream):
+            for d in self.sets:
+                fn(d)  # warm the library's per-device caches and the kernels before capture
+            self.stream.synchronize()
+            for d in self.sets:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=self.stream):
+                    fn(d)
+                gs.append(g)
+            self.stream.synchronize()
+        self.graphs[name] = gs
+        return gs
+
+    def release(self):
+        self.graphs.clear()
+        self.sets.clear()
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    from speculative_decoding_block_spec_b200 import synth
+    from speculative_decoding_block_spec_b200.dist import max_over_ranks as _max_over_ranks
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    stream = torch.cuda.Stream(dev)
+    peak, peak_src = measured_peaks()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
 
     def barrier():
         torch.cuda.synchronize(dev)
@@ -389,61 +530,8 @@ def main():
         """The slowest rank's time (the value itself on one GPU)."""
         return _max_over_ranks(ms, dev)
 
-    sampler = ClockSampler(local)
-    wall = {}
-    with torch.cuda.stream(stream):
-        t_w = time.time()
-        for i in range(args.warmup):
-            graphs[i % NSETS].replay()
-        barrier()
-        wall["warmup_s"] = time.time() - t_w
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        r0 = time.time()
-        e0.record(stream)
-        for i in range(args.steps):
-            graphs[i % NSETS].replay()
-        e1.record(stream)
-        e1.synchronize()
-        r1 = time.time()
-        sampler.region = (r0, r1)
-        wall["timed_s"] = r1 - r0
-        barrier()
-    sampler.stop()
-    ms_total = max_over_ranks(e0.elapsed_time(e1))
-    ms_step = ms_total / args.steps
-
-    # results of the last replay of set 0 give the bytes actually needed
-    acc = sets[0]["out"][0].cpu().numpy()
-    vl_np = sets[0]["dvl_out"][0].cpu().numpy() if w.budget is not None else np.full(w.B, w.L)
-    nbytes_step = step_bytes(w, vl_np, acc)
-    gbs_step = nbytes_step / (ms_step * 1e-3) / 1e9
-
-    # the dominant kernel alone: one verify launch (the DVL kernels, if any,
-    # already ran and their outputs stay fixed), one graph per input set
-    def verify_only(d):
-        vl = off = None
-        target = d["target"]
-        if w.budget is not None:
-            vl, off, target = d["dvl_out"][0], d["dvl_out"][1][:w.B], d["packed"]
-        if w.K == 1:
-            specv.spec_verify_block(target, d["draft"], d["tokens"], d["u"], d["g"], w.T, verify_len=vl,
-                                    target_row_off=off, workspace=d["ws"], out=d["out"])
-        else:
-            specv.spec_verify_mixture(target, d["draft"], d["mix_w"], d["tokens"], d["u"], d["g"], w.T,
-                                      verify_len=vl, target_row_off=off, workspace=d["ws"], out=d["out"])
-
-    def split_stages(d, stats_only=False):
-        vl = off = None
-        target = d["target"]
-        if w.budget is not None:
-            vl, off, target = d["dvl_out"][0], d["dvl_out"][1][:w.B], d["packed"]
-        specv.spec_verify_window_stats(target, d["draft"], d["tokens"], w.T, d["ws"], verify_len=vl,
-                                       target_row_off=off)
-        if not stats_only:
-            specv.spec_verify_accept(target, d["draft"], d["tokens"], d["u"], d["g"], w.T, d["ws"],
-                                     mix_w=d.get("mix_w"), verify_len=vl, target_row_off=off, out=d["out"])
-
-    def timed_loop(fn):
+    def timed_total(fn):
+        """W untimed calls, then K calls between one pair of events: ms per call (max over ranks)."""
         with torch.cuda.stream(stream):
             for i in range(args.warmup):
                 fn(i)
@@ -457,51 +545,106 @@ def main():
             barrier()
         return max_over_ranks(k0.elapsed_time(k1)) / args.steps
 
-    vgraphs, tgraphs = [], []
-    with torch.cuda.stream(stream):
-        for d in sets:
-            split_stages(d, stats_only=True)
-        stream.synchronize()
-        for d in sets:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                verify_only(d)
-            vgraphs.append(g)
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                split_stages(d, stats_only=True)
-            tgraphs.append(g)
-    ms_verify = timed_loop(lambda i: vgraphs[i % NSETS].replay())
-    ms_k = timed_loop(lambda i: tgraphs[i % NSETS].replay())
-    ms_pack = None
-    if w.budget is not None:  # allocation + pack copy, timed apart from the step
-        pgraphs = []
+    def timed_each(fn):
+        """W untimed calls, then K calls with one event pair each: their spread
+        (each statistic the max over ranks)."""
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
         with torch.cuda.stream(stream):
-            for d in sets:
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=stream):
-                    prepack(d)
-                pgraphs.append(g)
-        ms_pack = timed_loop(lambda i: pgraphs[i % NSETS].replay())
-        pgraphs.clear()
-    kb = window_bytes(w, vl_np)
-    peak, peak_src = measured_peaks()
-    achieved_k = kb / (ms_k * 1e-3) / 1e9
-    stats_kernel = stats_kernel_name(w, torch.cuda.get_device_properties(dev).multi_processor_count)
-    traffic, traffic_src = committed_traffic(stats_kernel, w.name)
+            for i in range(args.warmup):
+                fn(i)
+            barrier()
+            for i in range(args.steps):
+                ev[i][0].record(stream)
+                fn(i)
+                ev[i][1].record(stream)
+            stream.synchronize()
+            barrier()
+        s = spread([a.elapsed_time(b) for a, b in ev])
+        for k in ("median_ms", "p10_ms", "p90_ms", "min_ms", "max_ms"):
+            s[k] = max_over_ranks(s[k])
+        return s
 
-    # end to end: pinned host inputs -> device -> verify -> results to host
-    e2e = None
-    if not args.no_e2e:
+    def measure(cid, headline):
+        w = synth.WORKLOADS[cid]
+        x = synth.make_inputs(w, seed=rank)  # weak scaling: every rank verifies its own batch
+        r = Runner(w, x, dev, stream, args.sets)
+        ns = len(r.sets)
+        if w.budget is not None:
+            r.capture("pack", r.prepack)
+        graphs = r.capture("step", r.step)
+        res = {"w": w, "x": x}
+        sampler = ClockSampler(local) if headline else None
+        wall = {}
+        with torch.cuda.stream(stream):
+            t_w = time.time()
+            for i in range(args.warmup):
+                graphs[i % ns].replay()
+            barrier()
+            wall["warmup_s"] = time.time() - t_w
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            r0 = time.time()
+            e0.record(stream)
+            for i in range(args.steps):
+                graphs[i % ns].replay()
+            e1.record(stream)
+            e1.synchronize()
+            r1 = time.time()
+            wall["timed_s"] = r1 - r0
+            barrier()
+        if sampler is not None:
+            sampler.region = (r0, r1)
+            sampler.stop()
+            res["clocks"] = sampler.report()
+        res["wall"] = wall
+        ms_step = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+        res["ms_step"] = ms_step
+
+        # the outputs of the last replay of set 0 give the bytes actually needed
+        d0 = r.sets[0]
+        acc = d0["out"][0].cpu().numpy()
+        outt = d0["out"][1].cpu().numpy()
+        vl_np = d0["dvl_out"][0].cpu().numpy() if w.budget is not None else np.full(w.B, w.L)
+        res["gpu_out"] = (acc, outt)
+        res["step_bytes"] = step_bytes(w, vl_np, acc)
+
+        # replay by replay: the captured step, and the same step as plain launches
+        res["graph_replay"] = timed_each(lambda i: graphs[i % ns].replay())
+        res["plain_launch"] = timed_each(lambda i: r.step(r.sets[i % ns]))
+
+        # the verify call alone, and the statistics kernel alone (the roofline's kernel)
+        vg = r.capture("verify", r.verify_only)
+        res["ms_verify"] = timed_total(lambda i: vg[i % ns].replay())
+        tg = r.capture("stats", r.stats_only)
+        res["ms_stats"] = timed_total(lambda i: tg[i % ns].replay())
+        res["window_bytes"] = window_bytes(w, vl_np)
+        res["stats_kernel"] = stats_kernel_name(w, sms)
+        res["ms_pack"] = None
+        if w.budget is not None:  # allocation + pack copy, timed apart from the step
+            pg = r.graphs["pack"]
+            res["ms_pack"] = timed_total(lambda i: pg[i % ns].replay())
+
+        if headline and not args.no_e2e:
+            res["e2e"] = e2e_leg(r)
+        if not headline:
+            res["x"] = None  # only the headline's inputs feed the CPU baseline
+        r.release()
+        torch.cuda.empty_cache()
+        return res
+
+    def e2e_leg(r):
+        """End to end: pinned host inputs -> device -> verify through the public
+        API -> results to host, every step inside the timed region."""
+        w, x = r.w, r.x
         # with a DVL budget the target arrives as the packed rows the model produced
-        tgt = ("packed", sets[0]["packed"].cpu().pin_memory()) if w.budget is not None else \
+        tgt = ("packed", r.sets[0]["packed"].cpu().pin_memory()) if w.budget is not None else \
             ("target", torch.from_numpy(np.ascontiguousarray(x.target).view(
                 np.int16 if x.target.dtype == np.uint16 else np.float32)).pin_memory())
         host = dict([tgt],
-            draft=torch.from_numpy(np.ascontiguousarray(x.draft).view(
-                np.int16 if x.draft.dtype == np.uint16 else np.float32)).pin_memory(),
-            tokens=torch.from_numpy(x.tokens).pin_memory(), u=torch.from_numpy(x.u).pin_memory(),
-            g=torch.from_numpy(x.g).pin_memory())
+                    draft=torch.from_numpy(np.ascontiguousarray(x.draft).view(
+                        np.int16 if x.draft.dtype == np.uint16 else np.float32)).pin_memory(),
+                    tokens=torch.from_numpy(x.tokens).pin_memory(), u=torch.from_numpy(x.u).pin_memory(),
+                    g=torch.from_numpy(x.g).pin_memory())
         if x.mix_w is not None:
             host["mix_w"] = torch.from_numpy(x.mix_w).pin_memory()
         if x.scores is not None:
@@ -510,65 +653,84 @@ def main():
         res_acc = torch.empty(w.B, dtype=torch.int32).pin_memory()
         res_out = torch.empty((w.B, w.L + 1), dtype=torch.int32).pin_memory()
         d2h = res_acc.numel() * 4 + res_out.numel() * 4
-        n_e2e = min(args.steps, 50)
+        n_e2e = min(args.steps, 20)
+        ns = len(r.sets)
 
         def e2e_step(d):
             for k, t in host.items():
                 dst = d[k]
                 (dst.view(t.dtype) if dst.dtype != t.dtype else dst).copy_(t, non_blocking=True)
-            a, o = step(d)
+            a, o = r.step(d)
             res_acc.copy_(a, non_blocking=True)
             res_out.copy_(o, non_blocking=True)
 
         with torch.cuda.stream(stream):
             for i in range(3):
-                e2e_step(sets[i % NSETS])
+                e2e_step(r.sets[i % ns])
             barrier()
             t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             t0.record(stream)
             for i in range(n_e2e):
-                e2e_step(sets[i % NSETS])
+                e2e_step(r.sets[i % ns])
             t1.record(stream)
             t1.synchronize()
             barrier()
         ms_e2e = max_over_ranks(t0.elapsed_time(t1)) / n_e2e
-        e2e = {"value": world * w.B / (ms_e2e * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "steps": n_e2e,
-               "note": "pinned host inputs copied to HBM, verify through the public API, results read back"}
+        return {"value": world * w.B / (ms_e2e * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": n_e2e,
+                "note": "pinned host inputs copied to HBM, verify through the public API, results read back"}
 
-    cpu = None
+    def summary(res):
+        w = res["w"]
+        achieved = res["window_bytes"] / (res["ms_stats"] * 1e-3) / 1e9
+        gbs = res["step_bytes"] / (res["ms_step"] * 1e-3) / 1e9
+        traffic, traffic_src = committed_traffic(res["stats_kernel"], w.name)
+        return {
+            "value": world * w.B / (res["ms_step"] * 1e-3), "ms_per_step": res["ms_step"],
+            "hbm_gbs": gbs, "hbm_frac_of_nominal_8tbs": gbs / NOMINAL_HBM_GBS, "hbm_frac_of_measured_copy": gbs / peak,
+            "algorithmic_bytes_per_step": res["step_bytes"],
+            "roofline": {"bound": "hbm", "kernel": res["stats_kernel"], "achieved": achieved, "peak": peak,
+                         "unit": "GB/s", "frac": achieved / peak, "traffic": traffic, "traffic_source": traffic_src,
+                         "algorithmic_bytes_per_launch": res["window_bytes"], "launch_ms": res["ms_stats"],
+                         "peak_source": peak_src, "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
+                         "timed": "spec_verify_window_stats alone, CUDA graph replay over the rotating sets"},
+            "verify_ms": res["ms_verify"], "dvl_allocate_pack_ms": res["ms_pack"],
+            "per_replay": {"graph_replay": res["graph_replay"], "plain_launch": res["plain_launch"],
+                           "launch_gap_saving_us": (res["plain_launch"]["median_ms"] -
+                                                    res["graph_replay"]["median_ms"]) * 1e3,
+                           "note": "one event pair per step; plain = the same step as stream launches "
+                                   "through the Python binding"},
+        }
+
+    head = measure(args.workload, headline=True)
+    extras = [measure(c, headline=False) for c in args.extra_ids]
+
+    cpu = margins = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(x, args.cpu_seconds)
+        cpu, margins = cpu_baseline(head["x"], args.cpu_seconds, head["gpu_out"])
 
-    graphs.clear()
-    vgraphs.clear()
-    tgraphs.clear()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return 0
+    w = head["w"]
+    s = summary(head)
     line = {
-        "metric": METRIC, "value": world * w.B / (ms_step * 1e-3), "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "metric": METRIC, "value": s["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": s["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic (seeded per rank; Qwen3-size vocabulary, block 16)",
-        "config": {"workload": w.name, "B": w.B, "L": w.L, "V": w.V, "K": w.K, "T": w.T, "budget": w.budget,
-                   "l2": "%d rotating input sets of %.0f MB (> 126 MB L2 together)" % (NSETS, set_bytes / 1e6),
-                   "launch": "CUDA graph replay, %d launches per step" % launches_per_step,
-                   "parallelism": "dp%d" % world},
-        "hbm_gbs": gbs_step, "hbm_frac_of_nominal_8tbs": gbs_step / NOMINAL_HBM_GBS,
-        "hbm_frac_of_measured_copy": gbs_step / peak, "algorithmic_bytes_per_step": nbytes_step,
-        "roofline": {"bound": "hbm", "kernel": stats_kernel, "achieved": achieved_k, "peak": peak, "unit": "GB/s",
-                     "frac": achieved_k / peak, "traffic": traffic, "traffic_source": traffic_src,
-                     "algorithmic_bytes_per_launch": kb, "launch_ms": ms_k, "peak_source": peak_src,
-                     "frac_of_nominal_8tbs": achieved_k / NOMINAL_HBM_GBS,
-                     "timed": "spec_verify_window_stats alone, CUDA graph replay over the rotating sets"},
-        "verify_ms": ms_verify,
-        "dvl_allocate_pack_ms": ms_pack,
-        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
-        "clocks": sampler.report(), "host_wall_s": wall,
+        "config": config_of(w, args.sets, world),
+        "launch": "CUDA graph replay, %d launches per step" % ((2 if w.L > 0 else 1) + (w.budget is not None)),
     }
+    line.update({k: v for k, v in s.items() if k not in ("value", "ms_per_step")})
+    line.update({
+        "low_margin_decisions": margins, "cpu_baseline": cpu, "e2e": head.get("e2e"),
+        "gpu_launches": ((2 if w.L > 0 else 1) + (w.budget is not None)) * args.steps,
+        "clocks": head["clocks"], "host_wall_s": head["wall"],
+        "workloads": {e["w"].name: dict(summary(e), config=config_of(e["w"], args.sets, world)) for e in extras},
+    })
     print(json.dumps(line), flush=True)
     return 0
 

@@ -119,8 +119,11 @@ int spec_softmax_T(const void* logits, int dtype, int64_t rows, int64_t V, int64
  *         SPEC_ERR_UNSUPPORTED before anything is launched.
  * Set-up: the first call on a device looks up the array's device address with
  * cudaGetSymbolAddress, with that device current (the current device must be
- * the stream's device); a failed lookup returns SPEC_ERR_CUDA. Make that first
- * call on each device before any stream capture begins.
+ * the stream's device), and caches it under the id of the current CUDA
+ * context; a failed lookup returns SPEC_ERR_CUDA. Make that first call on
+ * each device before any stream capture begins. A device reset ends the
+ * context, so the first call after it looks the address up again (again
+ * outside any capture).
  * Sharing: every call on a device uses the same array. Nothing in it has to
  * start at zero (each call writes every slot before it reads it), but calls
  * whose kernels overlap on the GPU (different streams, or different host

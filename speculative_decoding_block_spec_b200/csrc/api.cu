@@ -5,6 +5,8 @@
 #include <cmath>
 #include <mutex>
 
+#include <cuda.h>  // driver API types only (no driver functions are linked)
+
 #include "specv.h"
 #include "common.cuh"
 #include "internal.h"
@@ -39,21 +41,65 @@ int sm_count() {
 // workspace after its header). Shared by every call on a device.
 static __device__ __align__(256) float2 g_noalloc_part[kGMax + SPEC_NOALLOC_MAX_ROWS];
 
-// Device address of g_noalloc_part on the current device, looked up once per
-// device (with that device current) and cached.
+// Id of the current CUDA context, unique over the life of the process (0 if
+// there is none yet or the driver cannot say). The two driver functions are
+// fetched through the runtime, so the library does not link the driver.
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 4000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(f);
+    f = nullptr;
+    q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(f);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of g_noalloc_part in the current context: looked up with
+// cudaGetSymbolAddress once per context (a device's primary context, with
+// that device current) and cached under the context's id. A device reset
+// ends the context, and the next call looks the address up again in the new
+// one. If the context id is unavailable the address is looked up every call.
 int noalloc_scratch(float2** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return SPEC_ERR_CUDA;
-  if (dev < 0 || dev >= 64) return SPEC_ERR_UNSUPPORTED;
+  struct Entry {
+    unsigned long long ctx;
+    void* ptr;
+  };
   static std::mutex mu;
-  static void* cache[64] = {};
-  std::lock_guard<std::mutex> lock(mu);
-  if (!cache[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_part) != cudaSuccess || !p) return SPEC_ERR_CUDA;
-    cache[dev] = p;
+  static Entry cache[64] = {};
+  static int next = 0;
+  const unsigned long long id = current_context_id();
+  if (id) {
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry& e : cache)
+      if (e.ctx == id) {
+        *out = static_cast<float2*>(e.ptr);
+        return SPEC_OK;
+      }
   }
-  *out = static_cast<float2*>(cache[dev]);
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_part) != cudaSuccess || !p) return SPEC_ERR_CUDA;
+  const unsigned long long id2 = id ? id : current_context_id();  // the lookup may have created the context
+  if (id2) {
+    std::lock_guard<std::mutex> lock(mu);
+    cache[next] = Entry{id2, p};
+    next = (next + 1) % 64;
+  }
+  *out = static_cast<float2*>(p);
   return SPEC_OK;
 }
 

@@ -41,6 +41,60 @@ def test_stats_kernel_choice_mirrors_the_library():
     assert bench.stats_kernel_name(odd, 148) == "k_row_stats"  # rows not 16-byte vectors
 
 
+def test_headline_is_the_largest_workload_and_extras_follow():
+    a = bench.parse_args([])
+    assert a.workload == 5 and synth.WORKLOADS[a.workload].name == "stress B64 L16 V151936 K4 bf16 budget544"
+    assert a.extra_ids == [2, 3, 4]
+    assert bench.parse_args(["--extras", ""]).extra_ids == []
+    assert bench.parse_args(["--workload", "3", "--extras", "2,3"]).extra_ids == [2]
+
+
+def test_both_arms_describe_the_workload_alike():
+    w = synth.WORKLOADS[5]
+    c = bench.config_of(w, 4, 1)
+    assert c["workload"] == w.name and c["budget"] == 544 and c["parallelism"] == "dp1"
+    assert "above the 126 MB L2" in c["l2"]
+    # one input set: target 64x17 rows + packed 544 rows + draft 64x4x16 rows (bf16), Gumbel 64x17 rows (fp32)
+    V = w.V
+    expect = 64 * 17 * V * 2 + 544 * V * 2 + 64 * 4 * 16 * V * 2 + 64 * 17 * V * 4 + 64 * 16 * 8 + 64 * 4 * 4 \
+        + 64 * 16 * 4
+    assert bench.set_bytes(w) == expect
+    assert "NOT above" in bench.l2_note(synth.WORKLOADS[1], 4)
+
+
+def test_spread():
+    s = bench.spread([3.0, 1.0, 2.0, 5.0, 4.0])
+    assert s["median_ms"] == 3.0 and s["min_ms"] == 1.0 and s["max_ms"] == 5.0 and s["n"] == 5
+    assert s["p10_ms"] <= s["median_ms"] <= s["p90_ms"]
+
+
+def _ref(acc, out, margins, gaps, kappas):
+    return {"accept_len": np.array(acc), "out_tokens": np.array(out), "accept_margin": np.array(margins),
+            "argmax_gap": np.array(gaps), "argmax_kappa": np.array(kappas)}
+
+
+def test_margin_report_counts_decisions_and_low_margins():
+    # two requests, L = 3: request 0 rejects at 1 (2 accept tests + draw), request 1 accepts all (3 + draw)
+    ref = _ref([1, 3], [[7, 9, -1, -1], [1, 2, 3, 4]], [[0.3, 0.2, 0.1], [0.5, 0.5, 0.5]], [1.0, 2.0], [1.0, 1.0])
+    acc = np.array([1, 3])
+    out = np.array([[7, 9, -1, -1], [1, 2, 3, 4]])
+    r = bench.margin_report(acc, out, ref, None)
+    assert r["decisions"] == 3 + 4 and r["low_margin"] == 0 and r["mismatches"] == 0
+    out2 = out.copy()
+    out2[1, 3] = 5
+    assert bench.margin_report(acc, out2, ref, None)["mismatches"] == 1
+    # the same difference under a low-margin terminal draw is exempt
+    ref_low = dict(ref, argmax_gap=np.array([1.0, 1e-8]))
+    r = bench.margin_report(acc, out2, ref_low, None)
+    assert r["low_margin"] == 1 and r["exempted_differences"] == 1 and r["mismatches"] == 0
+    # a low-margin accept test exempts the request's later outputs
+    ref_acc = dict(ref, accept_margin=np.array([[0.3, 5e-7, 0.1], [0.5, 0.5, 0.5]]))
+    acc3 = np.array([2, 3])
+    out3 = np.array([[7, 8, 6, -1], [1, 2, 3, 4]])
+    r = bench.margin_report(acc3, out3, ref_acc, None)
+    assert r["low_margin"] == 1 and r["exempted_differences"] == 1 and r["mismatches"] == 0
+
+
 def test_committed_traffic_needs_matching_source(tmp_path, monkeypatch):
     src = tmp_path / "k.cu"
     src.write_text("kernel source v1\n")
@@ -83,4 +137,4 @@ def test_reference_leg_prints_one_json_line():
     assert d["value"] > 0 and d["steps"] == 2 and d["warmup"] == 3
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
-    assert d["config"]["workload"] == synth.WORKLOADS[1].name
+    assert d["config"] == bench.config_of(synth.WORKLOADS[1], 4, 1)

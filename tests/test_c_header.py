@@ -63,5 +63,7 @@ def test_header_compiles_as_c_and_host_calls_behave(tmp_path):
                         "-L", lib_dir, "-lspecv", "-Wl,-rpath," + lib_dir, "-o", str(exe)],
                        capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
-    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    # no visible GPU: every call is rejected on the host, and one that were not could not launch
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120,
+                       env=dict(os.environ, CUDA_VISIBLE_DEVICES=""))
     assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)

@@ -3,8 +3,9 @@
 Every input is seeded and synthetic (speculative_decoding_block_spec_b200.synth).
 Decisions (accepted lengths, tokens, verify lengths, offsets, slot maps,
 packed rows) must match bit for bit, under the low-margin rule of
-tests/parity_util.py; softmax maxima, normalisers and probabilities within
-1e-5 relative.
+tests/parity_util.py (run-wide exemption budget); softmax maxima, normalisers
+and probabilities within 1e-5 relative (a normaliser through its log:
+|lse_gpu - lse_oracle| <= 1e-5).
 """
 import numpy as np
 import pytest
@@ -15,7 +16,7 @@ import speculative_decoding_block_spec_b200 as specv
 from speculative_decoding_block_spec_b200 import synth
 from speculative_decoding_block_spec_b200.synth import f32_to_bf16_bits
 
-from parity_util import check_verify, logits_to_torch, to_torch
+from parity_util import assert_softmax_close, check_verify, logits_to_torch, to_torch
 
 pytestmark = pytest.mark.gpu
 NT = oracle.n_cores()
@@ -45,7 +46,8 @@ def _cpu(t):
     (5, 1001, "bf16", 0.7, True),       # scalar path
     (1, 8, "bf16", 1.0, True),
     (300, 4096, "bf16", 1.0, True),     # many rows per block
-    (40, 151936, "bf16", 1.0, False),
+    (40, 151936, "bf16", 1.0, False),   # balanced one-block-per-SM kernel (5,133 units per SM)
+    (40, 151936, "bf16", 1.3, True),    # the same kernel, with probabilities
     (12, 151936, "bf16", 1.5, True),
     (3, 151936, "f32", 1.0, True),
 ])
@@ -57,10 +59,7 @@ def test_softmax_parity(rows, V, dtype, T, probs):
     xs = f32_to_bf16_bits(x) if dtype == "bf16" else x
     ref = oracle.softmax_T(xs, T, probs=probs)
     got = specv.softmax_T(logits_to_torch(xs), T, probs=probs)
-    np.testing.assert_allclose(_cpu(got[0]), ref[0], rtol=1e-5, atol=0)
-    np.testing.assert_allclose(_cpu(got[1]), ref[1], rtol=1e-5, atol=1e-6)
-    if probs:
-        np.testing.assert_allclose(_cpu(got[2]), ref[2], rtol=1e-5, atol=1e-37)
+    assert_softmax_close([_cpu(t) for t in got], ref)
 
 
 @pytest.mark.parametrize("dtype,V,stride", [("bf16", 4000, 4096), ("bf16", 4000, 4003), ("f32", 1000, 1024)])
@@ -84,9 +83,7 @@ def test_softmax_padded_row_stride(dtype, V, stride):
                                     rmax.data_ptr(), rlse.data_ptr(), probs.data_ptr(), ws.ptr(), ws.nbytes,
                                     torch.cuda.current_stream().cuda_stream)
     assert st == 0
-    np.testing.assert_allclose(_cpu(rmax), ref[0], rtol=1e-5, atol=0)
-    np.testing.assert_allclose(_cpu(rlse), ref[1], rtol=1e-5, atol=1e-6)
-    np.testing.assert_allclose(_cpu(probs), ref[2], rtol=1e-5, atol=1e-37)
+    assert_softmax_close([_cpu(rmax), _cpu(rlse), _cpu(probs)], ref)
 
 
 @pytest.mark.parametrize("K", [1, 3])
