@@ -63,6 +63,8 @@ def parse_args(argv=None):
     ap.add_argument("--extras", default="2,3,4",
                     help="comma-separated further workloads measured in the same run ('' for none)")
     ap.add_argument("--sets", type=int, default=4, help="rotating input sets (together above the L2 size)")
+    ap.add_argument("--top-p-extras", default="3", help="workloads also measured with top-p filtering ('' for none)")
+    ap.add_argument("--top-p", type=float, default=0.95, help="top-p of the filtered measurements")
     ap.add_argument("--impl", default="specv", choices=["specv", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU-baseline sample")
     ap.add_argument("--no-e2e", action="store_true")
@@ -70,6 +72,7 @@ def parse_args(argv=None):
     args = ap.parse_args(argv)
     args.extra_ids = [int(c) for c in args.extras.split(",") if c.strip()] if args.extras else []
     args.extra_ids = [c for c in args.extra_ids if c != args.workload]
+    args.top_p_ids = [int(c) for c in args.top_p_extras.split(",") if c.strip()] if args.top_p_extras else []
     return args
 
 
@@ -395,11 +398,12 @@ class Runner:
     """Device-side state of one workload: its rotating input sets, the step
     through the public API, and the CUDA graphs that replay it."""
 
-    def __init__(self, w, x, dev, stream, nsets):
+    def __init__(self, w, x, dev, stream, nsets, top_p=1.0):
         import torch
         import speculative_decoding_block_spec_b200 as specv
         self.torch, self.specv = torch, specv
         self.w, self.x, self.dev, self.stream = w, x, dev, stream
+        self.top_p = top_p
 
         def logits(a):
             if a.dtype == np.uint16:
@@ -420,7 +424,8 @@ class Runner:
                     d["dvl_out"] = (torch.empty(w.B, dtype=torch.int32, device=dev),
                                     torch.empty(w.B + 1, dtype=torch.int32, device=dev),
                                     torch.empty(w.budget, dtype=torch.int32, device=dev))
-                d["ws"] = specv.Workspace(specv.verify_workspace_size(w.B, w.L, w.K, w.V), dev)
+                d["ws"] = specv.Workspace(specv.verify_top_p_workspace_size(w.B, w.L, w.K, w.V) if top_p < 1 else
+                                          specv.verify_workspace_size(w.B, w.L, w.K, w.V), dev)
                 d["out"] = (torch.empty(w.B, dtype=torch.int32, device=dev),
                             torch.empty((w.B, w.L + 1), dtype=torch.int32, device=dev))
                 self.sets.append(d)
@@ -439,7 +444,8 @@ class Runner:
     def step(self, d):
         """One verify step through the public API (the launches a user makes):
         with a DVL budget, the allocation over the survival scores, then
-        verification of the packed rows at the allocated offsets."""
+        verification of the packed rows at the allocated offsets; with top-p,
+        the filtered verification."""
         w, specv = self.w, self.specv
         vl = off = None
         target = d["target"]
@@ -447,6 +453,14 @@ class Runner:
             vl, off, _ = specv.dvl_allocate_pack(d["scores"], w.budget, workspace=d["dvl_ws"], out=d["dvl_out"])
             off = off[:w.B]
             target = d["packed"]
+        if self.top_p < 1:
+            if w.K == 1:
+                return specv.spec_verify_block_top_p(target, d["draft"], d["tokens"], d["u"], d["g"], w.T,
+                                                     self.top_p, verify_len=vl, target_row_off=off,
+                                                     workspace=d["ws"], out=d["out"])
+            return specv.spec_verify_mixture_top_p(target, d["draft"], d["mix_w"], d["tokens"], d["u"], d["g"], w.T,
+                                                   self.top_p, verify_len=vl, target_row_off=off, workspace=d["ws"],
+                                                   out=d["out"])
         if w.K == 1:
             return specv.spec_verify_block(target, d["draft"], d["tokens"], d["u"], d["g"], w.T, verify_len=vl,
                                            target_row_off=off, workspace=d["ws"], out=d["out"])
@@ -565,10 +579,23 @@ def main(argv=None):
             s[k] = max_over_ranks(s[k])
         return s
 
-    def measure(cid, headline):
+    def measure(cid, headline, top_p=1.0):
         w = synth.WORKLOADS[cid]
         x = synth.make_inputs(w, seed=rank)  # weak scaling: every rank verifies its own batch
-        r = Runner(w, x, dev, stream, args.sets)
+        r = Runner(w, x, dev, stream, args.sets, top_p)
+        if top_p < 1:  # the filtered step alone: statistics with bonus rows, nuclei, accept / sample
+            graphs = r.capture("step", r.step)
+            ns = len(r.sets)
+            res = {"w": w, "x": None, "top_p": top_p}
+            res["ms_step"] = timed_total(lambda i: graphs[i % ns].replay())
+            res["graph_replay"] = timed_each(lambda i: graphs[i % ns].replay())
+            acc = r.sets[0]["out"][0].cpu().numpy()
+            res["flagged_requests"] = int((acc < 0).sum())
+            vl_np = np.full(w.B, w.L)
+            res["step_bytes"] = step_bytes(w, vl_np, acc) + w.B * w.V * (2 if w.dtype == "bf16" else 4)
+            r.release()
+            torch.cuda.empty_cache()
+            return res
         ns = len(r.sets)
         if w.budget is not None:
             r.capture("pack", r.prepack)
@@ -704,6 +731,7 @@ def main(argv=None):
 
     head = measure(args.workload, headline=True)
     extras = [measure(c, headline=False) for c in args.extra_ids]
+    filtered = [measure(c, headline=False, top_p=args.top_p) for c in args.top_p_ids]
 
     cpu = margins = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -730,6 +758,15 @@ def main(argv=None):
         "gpu_launches": ((2 if w.L > 0 else 1) + (w.budget is not None)) * args.steps,
         "clocks": head["clocks"], "host_wall_s": head["wall"],
         "workloads": {e["w"].name: dict(summary(e), config=config_of(e["w"], args.sets, world)) for e in extras},
+        "top_p_workloads": {"%s top_p %g" % (f["w"].name, f["top_p"]): {
+            "value": world * f["w"].B / (f["ms_step"] * 1e-3), "unit": UNIT, "ms_per_step": f["ms_step"],
+            "top_p": f["top_p"], "graph_replay": f["graph_replay"], "flagged_requests": f["flagged_requests"],
+            "algorithmic_bytes_per_step": f["step_bytes"],
+            "hbm_gbs_algorithmic": f["step_bytes"] / (f["ms_step"] * 1e-3) / 1e9,
+            "note": "spec_verify_*_top_p (statistics with bonus rows, nucleus kernel, accept / sample); "
+                    "drafted tokens from the seeded generator, i.e. from the unfiltered draft rows; algorithmic "
+                    "bytes count each filtered row once, as the unfiltered step does, plus the bonus rows"}
+            for f in filtered},
     })
     print(json.dumps(line), flush=True)
     return 0

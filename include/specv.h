@@ -200,6 +200,54 @@ int spec_verify_mixture(const void* target_logits, const int32_t* target_row_off
                         void* workspace, size_t ws_bytes, spec_stream_t stream);
 
 /*
+ * spec_verify_block_top_p, spec_verify_mixture_top_p — the same
+ * verification with every row filtered to its top-p nucleus ([DBLAST]
+ * "What would settle it": target sampling at T = 1.5 with top-p 0.95;
+ * "Assumptions": target probabilities under the same sampling filter, here
+ * applied to the target rows and to every draft category alike).
+ * The nucleus of a row (temperature softmax of x / T) is the shortest run of
+ * its tokens, ordered by probability descending and index ascending, whose
+ * probability mass reaches top_p; kept tokens are renormalised by that mass
+ * and every other token has probability 0. Then, as in spec_verify_block /
+ * spec_verify_mixture with the filtered rows:
+ *   a drafted token outside target row i's nucleus is rejected (p = 0);
+ *   one that the filtered proposal gives probability 0 is accepted;
+ *   the residual max(0, p_j - q_j) and the bonus row l are the filtered ones.
+ * A request whose accepted tokens have probability 0 under every filtered
+ * draft category (impossible when the drafts were sampled from the filtered
+ * proposal) has no posterior: SPEC_DEV_NONFINITE, accept_len = -1.
+ *   top_p      in (0, 1]; 1 is the unfiltered call (same results as
+ *              spec_verify_block / spec_verify_mixture); NaN or <= 0:
+ *              SPEC_ERR_ARG.
+ *   workspace  >= spec_verify_top_p_workspace_size(B, L, K, V) bytes, zeroed
+ *              once (it also serves the unfiltered calls of the same shape).
+ * Other arguments and limits as spec_verify_block / spec_verify_mixture
+ * (K = 1 and w = 1 for the block variant).
+ * Execution: three launches chained with programmatic dependent launch:
+ * the statistics of the verify window plus each request's bonus row; a
+ * nucleus kernel that finds each row's cut (a radix descent over the
+ * logits' order keys with exact fixed-point masses, then the tie cut by
+ * token index); the accept / sample stage with the filtered rows.
+ */
+size_t spec_verify_top_p_workspace_size(int B, int L, int K, int64_t V);
+
+int spec_verify_block_top_p(const void* target_logits, const int32_t* target_row_off,
+                            const void* draft_logits, int dtype,
+                            const int32_t* draft_tokens, const int32_t* verify_len,
+                            const float* uniforms, const float* gumbel,
+                            int B, int L, int64_t V, float T, float top_p,
+                            int32_t* accept_len, int32_t* out_tokens,
+                            void* workspace, size_t ws_bytes, spec_stream_t stream);
+
+int spec_verify_mixture_top_p(const void* target_logits, const int32_t* target_row_off,
+                              const void* draft_logits, const float* mix_weights, int K, int dtype,
+                              const int32_t* draft_tokens, const int32_t* verify_len,
+                              const float* uniforms, const float* gumbel,
+                              int B, int L, int64_t V, float T, float top_p,
+                              int32_t* accept_len, int32_t* out_tokens,
+                              void* workspace, size_t ws_bytes, spec_stream_t stream);
+
+/*
  * The two stages that spec_verify_block / spec_verify_mixture launch, for
  * callers that schedule them separately (e.g. to time or overlap them).
  *
@@ -238,7 +286,8 @@ int spec_verify_accept(const void* target_logits, const int32_t* target_row_off,
  * dvl_allocate_pack — dynamic verify-length allocation ([DSCALE] Abstract;
  * [QA] prefix survival probabilities).
  *   scores        [B, L] fp32 per-position survival scores s[b,i] in [0, 1]
- *                 (outside: SPEC_DEV_SCORES, results unspecified but in range).
+ *                 (outside: SPEC_DEV_SCORES, results unspecified but in range;
+ *                 NULL allowed when L == 0).
  *   P[b,i] = s[b,0] * ... * s[b,i] in fp64, left to right (non-increasing in i).
  *   budget        total verify slots, >= B; slots used = min(budget, B*(L+1)).
  *                 Every request keeps its root slot; the other
@@ -257,6 +306,8 @@ int spec_verify_accept(const void* target_logits, const int32_t* target_row_off,
  * The outputs live at fixed addresses and feed spec_verify_* (verify_len,
  * target_row_off = offsets) on the device, so one captured graph serves
  * every allocation. Limits: B * L <= SPEC_MAX_DVL_ELEMS, L <= SPEC_MAX_L.
+ * Execution: one thread block; a radix select over the products' 64-bit
+ * keys finds the cut, so the work is O(B * L).
  */
 int dvl_allocate_pack(const float* scores, int B, int L, int budget,
                       int32_t* verify_len, int32_t* offsets, int32_t* slot_map,

@@ -13,6 +13,8 @@ Entry points (same names as the C ABI):
   spec_softmax_T_noalloc(logits, T, row_max, row_lse, probs=None)
   spec_verify_block(target, draft, tokens, u, g, T, ...)
   spec_verify_mixture(target, draft, mix_w, tokens, u, g, T, ...)
+  spec_verify_block_top_p(target, draft, tokens, u, g, T, top_p, ...)     rows filtered to their nuclei
+  spec_verify_mixture_top_p(target, draft, mix_w, tokens, u, g, T, top_p, ...)
   spec_verify_window_stats(...), spec_verify_accept(...)   the two verify stages
   dvl_allocate_pack(scores, budget, dense_target=None, packed_target=None)
 Workspaces: Workspace(nbytes, device), with verify/softmax/dvl size helpers;
@@ -24,7 +26,8 @@ import os
 import torch
 
 __all__ = ["SpecError", "Workspace", "lib", "softmax_T", "spec_softmax_T", "spec_softmax_T_noalloc", "NOALLOC_MAX_ROWS", "spec_verify_block",
-           "spec_verify_mixture", "spec_verify_window_stats", "spec_verify_accept", "dvl_allocate_pack", "verify_workspace_size", "softmax_workspace_size",
+           "spec_verify_mixture", "spec_verify_block_top_p", "spec_verify_mixture_top_p",
+           "verify_top_p_workspace_size", "spec_verify_window_stats", "spec_verify_accept", "dvl_allocate_pack", "verify_workspace_size", "softmax_workspace_size",
            "dvl_workspace_size", "check_verify_args", "LIB_PATH", "EXPORTS", "DEV_TOKEN_RANGE", "DEV_NONFINITE", "DEV_VERIFY_LEN",
            "DEV_SCORES"]
 
@@ -39,12 +42,16 @@ _SIGS = {
     "spec_status_string": ([_I], ctypes.c_char_p),
     "spec_softmax_workspace_size": ([_I64], _SZ),
     "spec_verify_workspace_size": ([_I, _I, _I, _I64], _SZ),
+    "spec_verify_top_p_workspace_size": ([_I, _I, _I, _I64], _SZ),
     "spec_dvl_workspace_size": ([_I], _SZ),
     "spec_workspace_init": ([_P, _SZ, _P], _I),
     "spec_softmax_T": ([_P, _I, _I64, _I64, _I64, _F, _P, _P, _P, _P, _SZ, _P], _I),
     "spec_softmax_T_noalloc": ([_P, _I, _I64, _I64, _I64, _F, _P, _P, _P, _P], _I),
     "spec_verify_block": ([_P, _P, _P, _I, _P, _P, _P, _P, _I, _I, _I64, _F, _P, _P, _P, _SZ, _P], _I),
     "spec_verify_mixture": ([_P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _I, _I, _I64, _F, _P, _P, _P, _SZ, _P], _I),
+    "spec_verify_block_top_p": ([_P, _P, _P, _I, _P, _P, _P, _P, _I, _I, _I64, _F, _F, _P, _P, _P, _SZ, _P], _I),
+    "spec_verify_mixture_top_p": ([_P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _I, _I, _I64, _F, _F, _P, _P, _P, _SZ, _P],
+                                  _I),
     "spec_verify_window_stats": ([_P, _P, _P, _I, _I, _P, _P, _I, _I, _I64, _F, _P, _SZ, _P], _I),
     "spec_verify_accept": ([_P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _I, _I, _I64, _F, _P, _P, _P, _SZ, _P], _I),
     "dvl_allocate_pack": ([_P, _I, _I, _I, _P, _P, _P, _P, _P, _I, _I64, _P, _SZ, _P], _I),
@@ -90,6 +97,10 @@ def softmax_workspace_size(rows):
 
 def verify_workspace_size(B, L, K=1, V=151936):
     return int(lib().spec_verify_workspace_size(B, L, K, V))
+
+
+def verify_top_p_workspace_size(B, L, K=1, V=151936):
+    return int(lib().spec_verify_top_p_workspace_size(B, L, K, V))
 
 
 def dvl_workspace_size(B):
@@ -280,6 +291,43 @@ def spec_verify_mixture(target, draft, mix_w, tokens, u, g, T, *, verify_len=Non
           _dev(draft, "draft"), _dev(mix_w, "mix_w", torch.float32), K, _dtype_code(draft),
           _dev(tokens, "tokens", torch.int32), _opt(verify_len, "verify_len", torch.int32),
           _dev(u, "u", torch.float32), _dev(g, "g", torch.float32), B, L, V, float(T),
+          _dev(acc, "accept_len", torch.int32), _dev(outt, "out_tokens", torch.int32), ws.ptr(), ws.nbytes,
+          _stream(draft))
+    return acc, outt
+
+
+def spec_verify_block_top_p(target, draft, tokens, u, g, T, top_p, *, verify_len=None, target_row_off=None,
+                            workspace=None, out=None):
+    """spec_verify_block with every target and draft row filtered to its top-p
+    nucleus (0 < top_p <= 1). The workspace is verify_top_p_workspace_size."""
+    B, L, _, V = check_verify_args(target, draft, tokens, u, g, verify_len=verify_len,
+                                   target_row_off=target_row_off, out=out, mixture=False)
+    ws = workspace or Workspace(verify_top_p_workspace_size(B, L, 1, V), draft.device)
+    acc, outt = _outputs(B, L, draft.device, out)
+    if _dtype_code(target) != _dtype_code(draft):
+        raise TypeError("target and draft logits must share a dtype")
+    _call("spec_verify_block_top_p", _dev(target, "target"), _opt(target_row_off, "target_row_off", torch.int32),
+          _dev(draft, "draft"), _dtype_code(draft), _dev(tokens, "tokens", torch.int32),
+          _opt(verify_len, "verify_len", torch.int32), _dev(u, "u", torch.float32), _dev(g, "g", torch.float32),
+          B, L, V, float(T), float(top_p), _dev(acc, "accept_len", torch.int32),
+          _dev(outt, "out_tokens", torch.int32), ws.ptr(), ws.nbytes, _stream(draft))
+    return acc, outt
+
+
+def spec_verify_mixture_top_p(target, draft, mix_w, tokens, u, g, T, top_p, *, verify_len=None,
+                              target_row_off=None, workspace=None, out=None):
+    """spec_verify_mixture with every target and draft row filtered to its
+    top-p nucleus (0 < top_p <= 1)."""
+    B, L, K, V = check_verify_args(target, draft, tokens, u, g, mix_w=mix_w, verify_len=verify_len,
+                                   target_row_off=target_row_off, out=out, mixture=True)
+    ws = workspace or Workspace(verify_top_p_workspace_size(B, L, K, V), draft.device)
+    acc, outt = _outputs(B, L, draft.device, out)
+    if _dtype_code(target) != _dtype_code(draft):
+        raise TypeError("target and draft logits must share a dtype")
+    _call("spec_verify_mixture_top_p", _dev(target, "target"), _opt(target_row_off, "target_row_off", torch.int32),
+          _dev(draft, "draft"), _dev(mix_w, "mix_w", torch.float32), K, _dtype_code(draft),
+          _dev(tokens, "tokens", torch.int32), _opt(verify_len, "verify_len", torch.int32),
+          _dev(u, "u", torch.float32), _dev(g, "g", torch.float32), B, L, V, float(T), float(top_p),
           _dev(acc, "accept_len", torch.int32), _dev(outt, "out_tokens", torch.int32), ws.ptr(), ws.nbytes,
           _stream(draft))
     return acc, outt

@@ -104,33 +104,48 @@ int noalloc_scratch(float2** out) {
 }
 
 // Resident sampling blocks per SM (cached per device and kernel variant).
-int accept_slots(int dtype, bool vec, int K) {
+int accept_slots(int dtype, bool vec, int K, bool topp) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
   static std::mutex mu;
-  static int cache[64][8] = {};
+  static int cache[64][16] = {};
   std::lock_guard<std::mutex> lock(mu);
-  int& c = cache[dev][dtype * 4 + (vec ? 2 : 0) + (K == 1 ? 1 : 0)];
-  if (!c) c = accept_blocks_per_sm(dtype, vec, K);
+  int& c = cache[dev][(topp ? 8 : 0) + dtype * 4 + (vec ? 2 : 0) + (K == 1 ? 1 : 0)];
+  if (!c) c = accept_blocks_per_sm(dtype, vec, K, topp);
   return c;
 }
 
 // Verify workspace: persistent state first (zero between calls), then scratch.
+// The walk has B (K+1) L rows, plus one bonus row per request with top-p
+// filtering, whose nucleus kernel adds four per-row arrays.
 struct VerifyLayout {
   size_t ticket, keys;     // persistent: per-request tickets [B], terminal keys [2B]
   size_t xg, rpart;        // scratch
+  size_t nm, nlf, nkey, nv;  // top-p scratch: row maxima, log nucleus masses, cut keys, cut tokens
   size_t total;
 };
 
-VerifyLayout verify_layout(int B, int L, int K, int64_t V) {
+size_t walk_rows(int B, int L, int K, bool topp) {
+  return static_cast<size_t>(B) * (static_cast<size_t>(K + 1) * L + (topp ? 1 : 0));
+}
+
+VerifyLayout verify_layout(int B, int L, int K, int64_t V, bool topp = false) {
   (void)V;
   VerifyLayout l;
-  const size_t rows = static_cast<size_t>(B) * (K + 1) * L;
+  const size_t rows = walk_rows(B, L, K, topp);
   l.ticket = kHeader;
   l.keys = l.ticket + align256(static_cast<size_t>(B) * sizeof(int));
   l.xg = l.keys + align256(static_cast<size_t>(2 * B) * sizeof(unsigned long long));
   l.rpart = l.xg + align256(rows * sizeof(float));
   l.total = l.rpart + align256((static_cast<size_t>(kGMax) + rows) * sizeof(float2));
+  l.nm = l.nlf = l.nkey = l.nv = 0;
+  if (topp) {
+    l.nm = l.total;
+    l.nlf = l.nm + align256(rows * sizeof(float));
+    l.nkey = l.nlf + align256(rows * sizeof(double));
+    l.nv = l.nkey + align256(rows * sizeof(uint32_t));
+    l.total = l.nv + align256(rows * sizeof(int32_t));
+  }
   return l;
 }
 
@@ -142,7 +157,7 @@ bool verify_shape_ok(int B, int L, int K) {
 int verify_check(const void* target, const int32_t* row_off, const void* draft, const float* mix_w, int K,
                  int dtype, const int32_t* tokens, const int32_t* vlen, const float* u, const float* g, int B, int L,
                  int64_t V, float T, const int32_t* accept_len, const int32_t* out_tokens, const void* ws,
-                 size_t ws_bytes, bool accept_stage) {
+                 size_t ws_bytes, bool accept_stage, bool topp = false) {
   // [B, L] and [B, K, L, V] arrays are empty when L == 0, so their pointers may then be NULL.
   if (!target || (L > 0 && !draft)) return SPEC_ERR_ARG;
   if (accept_stage && (!g || !accept_len || !out_tokens || (L > 0 && (!tokens || !u)))) return SPEC_ERR_ARG;
@@ -151,7 +166,7 @@ int verify_check(const void* target, const int32_t* row_off, const void* draft, 
   if (!verify_shape_ok(B, L, K) || V > SPEC_MAX_V) return SPEC_ERR_UNSUPPORTED;
   if (accept_stage && K > 1 && !mix_w) return SPEC_ERR_ARG;
   if (!ws) return SPEC_ERR_WORKSPACE;
-  if (ws_bytes < verify_layout(B, L, K, V).total) return SPEC_ERR_WORKSPACE;
+  if (ws_bytes < verify_layout(B, L, K, V, topp).total) return SPEC_ERR_WORKSPACE;
   const int es = esize(dtype);
   if (!aligned(target, es) || !aligned(draft, es) || !aligned(g, 4) || !aligned(u, 4) || !aligned(tokens, 4) ||
       !aligned(accept_len, 4) || !aligned(out_tokens, 4) || !aligned(ws, 16) || !aligned(row_off, 4) ||
@@ -166,37 +181,71 @@ bool stats_vec(const void* target, const void* draft, int dtype, int64_t V) {
   return (V * esize(dtype)) % 16 == 0 && aligned(target, 16) && aligned(draft, 16);
 }
 
-int launch_stats_stage(const void* target, const int32_t* row_off, const void* draft, int K, int dtype,
-                       const int32_t* tokens, const int32_t* vlen, int B, int L, int64_t V, float T, void* ws,
-                       cudaStream_t st) {
-  if (L == 0) return SPEC_OK;
-  const bool vec = stats_vec(target, draft, dtype, V);
-  const VerifyLayout lay = verify_layout(B, L, K, V);
+// The walk of the statistics stage (bonus rows with top-p filtering).
+RowSpace verify_walk(const void* target, const int32_t* row_off, const void* draft, int K, const int32_t* tokens,
+                     const int32_t* vlen, int B, int L, int64_t V, float* xg, bool topp) {
   RowSpace rs = {};
   rs.target = target;
   rs.draft = draft;
   rs.row_off = row_off;
   rs.vlen = vlen;
   rs.tokens = tokens;
-  rs.xg = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.xg);
+  rs.xg = xg;
   rs.stride = V;
   rs.rows = 0;
   rs.B = B;
   rs.L = L;
   rs.K = K;
   rs.verify = 1;
+  rs.bonus = topp ? 1 : 0;
+  return rs;
+}
+
+int stats_grid_of(int dtype, bool vec, int B, int L, int K, int64_t V, bool topp) {
   const int64_t Vu = units_per_row(V, dtype, vec);
-  const int G = stats_grid(dtype, vec, static_cast<int64_t>(B) * (K + 1) * L * Vu, Vu);
+  return stats_grid(dtype, vec, static_cast<int64_t>(walk_rows(B, L, K, topp)) * Vu, Vu);
+}
+
+int launch_stats_stage(const void* target, const int32_t* row_off, const void* draft, int K, int dtype,
+                       const int32_t* tokens, const int32_t* vlen, int B, int L, int64_t V, float T, void* ws,
+                       cudaStream_t st, bool topp = false) {
+  if (L == 0 && !topp) return SPEC_OK;
+  const bool vec = stats_vec(target, draft, dtype, V);
+  const VerifyLayout lay = verify_layout(B, L, K, V, topp);
+  RowSpace rs = verify_walk(target, row_off, draft, K, tokens, vlen, B, L, V,
+                            reinterpret_cast<float*>(static_cast<char*>(ws) + lay.xg), topp);
+  const int G = stats_grid_of(dtype, vec, B, L, K, V, topp);
   return map_cuda(launch_row_stats(rs, dtype, vec, V, T, G, reinterpret_cast<float2*>(static_cast<char*>(ws) + lay.rpart), st));
+}
+
+int launch_nucleus_stage(const void* target, const int32_t* row_off, const void* draft, int K, int dtype,
+                         const int32_t* tokens, const int32_t* vlen, int B, int L, int64_t V, float T, float top_p,
+                         void* ws, cudaStream_t st) {
+  const bool vec = stats_vec(target, draft, dtype, V);
+  const VerifyLayout lay = verify_layout(B, L, K, V, true);
+  char* w = static_cast<char*>(ws);
+  NucleusArgs a = {};
+  a.rs = verify_walk(target, row_off, draft, K, tokens, vlen, B, L, V, reinterpret_cast<float*>(w + lay.xg), true);
+  a.part = reinterpret_cast<const float2*>(w + lay.rpart);
+  a.G = stats_grid_of(dtype, vec, B, L, K, V, true);
+  a.Vu = units_per_row(V, dtype, vec);
+  a.V = V;
+  a.k = static_cast<float>(1.4426950408889634 / static_cast<double>(T));
+  a.top_p = static_cast<double>(top_p);
+  a.row_m = reinterpret_cast<float*>(w + lay.nm);
+  a.row_lf = reinterpret_cast<double*>(w + lay.nlf);
+  a.cut_key = reinterpret_cast<uint32_t*>(w + lay.nkey);
+  a.cut_v = reinterpret_cast<int32_t*>(w + lay.nv);
+  return map_cuda(launch_nucleus(a, dtype, vec, st));
 }
 
 int launch_accept_stage(const void* target, const int32_t* row_off, const void* draft, const float* mix_w, int K,
                         int dtype, const int32_t* tokens, const int32_t* vlen, const float* u, const float* g, int B,
                         int L, int64_t V, float T, int32_t* accept_len, int32_t* out_tokens, void* ws,
-                        cudaStream_t st) {
+                        cudaStream_t st, bool topp = false) {
   const bool vec = stats_vec(target, draft, dtype, V);
   const bool vec_term = vec && aligned(g, 16);
-  const VerifyLayout lay = verify_layout(B, L, K, V);
+  const VerifyLayout lay = verify_layout(B, L, K, V, topp);
   char* w = static_cast<char*>(ws);
   VerifyArgs a = {};
   a.target = target;
@@ -220,27 +269,42 @@ int launch_accept_stage(const void* target, const int32_t* row_off, const void* 
   a.xg = reinterpret_cast<const float*>(w + lay.xg);
   a.rpart = reinterpret_cast<const float2*>(w + lay.rpart);
   a.Vu = units_per_row(V, dtype, vec);
-  a.G = stats_grid(dtype, vec, static_cast<int64_t>(B) * (K + 1) * L * a.Vu, a.Vu);
+  a.G = stats_grid_of(dtype, vec, B, L, K, V, topp);
+  a.topp = topp ? 1 : 0;
+  if (topp) {
+    a.nuc_m = reinterpret_cast<const float*>(w + lay.nm);
+    a.nuc_lf = reinterpret_cast<const double*>(w + lay.nlf);
+    a.nuc_key = reinterpret_cast<const uint32_t*>(w + lay.nkey);
+    a.nuc_v = reinterpret_cast<const int32_t*>(w + lay.nv);
+  }
   // Blocks per request for the terminal row: the whole (P, B) grid resident
   // at once (no second wave), at least 256 units of the row per block.
   const int64_t term_units = vec_term ? V / (16 / esize(dtype)) : V;
-  const int64_t slots = static_cast<int64_t>(sm_count()) * accept_slots(dtype, vec_term, K);
+  const int64_t slots = static_cast<int64_t>(sm_count()) * accept_slots(dtype, vec_term, K, topp);
   const int64_t p_fit = std::max<int64_t>(1, slots / B);
   a.P = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({p_fit, kPMax, term_units / kThreads})));
   return map_cuda(launch_accept_sample(a, dtype, vec_term, st));
 }
 
+// top_p >= 1: unfiltered (two stages); below 1: statistics with bonus rows,
+// the nucleus kernel, then the filtered accept / sample stage.
 int verify_common(const void* target, const int32_t* row_off, const void* draft, const float* mix_w, int K,
                   int dtype, const int32_t* tokens, const int32_t* vlen, const float* u, const float* g, int B,
                   int L, int64_t V, float T, int32_t* accept_len, int32_t* out_tokens, void* ws, size_t ws_bytes,
-                  cudaStream_t st) {
+                  cudaStream_t st, float top_p = 1.f) {
+  if (!(top_p > 0.f && top_p <= 1.f)) return SPEC_ERR_ARG;  // NaN included
+  const bool topp = top_p < 1.f;
   int e = verify_check(target, row_off, draft, mix_w, K, dtype, tokens, vlen, u, g, B, L, V, T, accept_len,
-                       out_tokens, ws, ws_bytes, true);
+                       out_tokens, ws, ws_bytes, true, topp);
   if (e) return e;
-  e = launch_stats_stage(target, row_off, draft, K, dtype, tokens, vlen, B, L, V, T, ws, st);
+  e = launch_stats_stage(target, row_off, draft, K, dtype, tokens, vlen, B, L, V, T, ws, st, topp);
   if (e) return e;
+  if (topp) {
+    e = launch_nucleus_stage(target, row_off, draft, K, dtype, tokens, vlen, B, L, V, T, top_p, ws, st);
+    if (e) return e;
+  }
   return launch_accept_stage(target, row_off, draft, mix_w, K, dtype, tokens, vlen, u, g, B, L, V, T, accept_len,
-                             out_tokens, ws, st);
+                             out_tokens, ws, st, topp);
 }
 
 }  // namespace
@@ -266,6 +330,11 @@ size_t spec_softmax_workspace_size(int64_t rows) {
 size_t spec_verify_workspace_size(int B, int L, int K, int64_t V) {
   if (!verify_shape_ok(B, L, K) || V < 1 || V > SPEC_MAX_V) return 0;
   return verify_layout(B, L, K, V).total;
+}
+
+size_t spec_verify_top_p_workspace_size(int B, int L, int K, int64_t V) {
+  if (!verify_shape_ok(B, L, K) || V < 1 || V > SPEC_MAX_V) return 0;
+  return verify_layout(B, L, K, V, true).total;
 }
 
 size_t spec_dvl_workspace_size(int B) {
@@ -360,6 +429,27 @@ int spec_verify_mixture(const void* target_logits, const int32_t* target_row_off
                        reinterpret_cast<cudaStream_t>(stream));
 }
 
+int spec_verify_block_top_p(const void* target_logits, const int32_t* target_row_off, const void* draft_logits,
+                            int dtype, const int32_t* draft_tokens, const int32_t* verify_len, const float* uniforms,
+                            const float* gumbel, int B, int L, int64_t V, float T, float top_p,
+                            int32_t* accept_len, int32_t* out_tokens, void* workspace, size_t ws_bytes,
+                            spec_stream_t stream) {
+  return verify_common(target_logits, target_row_off, draft_logits, nullptr, 1, dtype, draft_tokens, verify_len,
+                       uniforms, gumbel, B, L, V, T, accept_len, out_tokens, workspace, ws_bytes,
+                       reinterpret_cast<cudaStream_t>(stream), top_p);
+}
+
+int spec_verify_mixture_top_p(const void* target_logits, const int32_t* target_row_off, const void* draft_logits,
+                              const float* mix_weights, int K, int dtype, const int32_t* draft_tokens,
+                              const int32_t* verify_len, const float* uniforms, const float* gumbel, int B, int L,
+                              int64_t V, float T, float top_p, int32_t* accept_len, int32_t* out_tokens,
+                              void* workspace, size_t ws_bytes, spec_stream_t stream) {
+  if (!mix_weights) return SPEC_ERR_ARG;
+  return verify_common(target_logits, target_row_off, draft_logits, mix_weights, K, dtype, draft_tokens, verify_len,
+                       uniforms, gumbel, B, L, V, T, accept_len, out_tokens, workspace, ws_bytes,
+                       reinterpret_cast<cudaStream_t>(stream), top_p);
+}
+
 int spec_verify_window_stats(const void* target_logits, const int32_t* target_row_off, const void* draft_logits,
                              int K, int dtype, const int32_t* draft_tokens, const int32_t* verify_len, int B, int L,
                              int64_t V, float T, void* workspace, size_t ws_bytes, spec_stream_t stream) {
@@ -388,8 +478,8 @@ int spec_verify_accept(const void* target_logits, const int32_t* target_row_off,
 int dvl_allocate_pack(const float* scores, int B, int L, int budget, int32_t* verify_len, int32_t* offsets,
                       int32_t* slot_map, const void* dense_target, void* packed_target, int dtype, int64_t V,
                       void* workspace, size_t ws_bytes, spec_stream_t stream) {
-  if (!scores || !verify_len || !offsets) return SPEC_ERR_ARG;
   if (B < 1 || L < 0 || budget < B) return SPEC_ERR_ARG;
+  if ((!scores && L > 0) || !verify_len || !offsets) return SPEC_ERR_ARG;  // [B, 0] scores may be NULL
   if (B > SPEC_MAX_B || L > SPEC_MAX_L || static_cast<int64_t>(B) * L > SPEC_MAX_DVL_ELEMS)
     return SPEC_ERR_UNSUPPORTED;
   const bool pack = dense_target || packed_target;
@@ -402,8 +492,7 @@ int dvl_allocate_pack(const float* scores, int B, int L, int budget, int32_t* ve
   if (ws_bytes < spec_dvl_workspace_size(B) || !aligned(workspace, 16)) return SPEC_ERR_WORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   int* status = static_cast<int*>(workspace);
-  int* ticket = reinterpret_cast<int*>(static_cast<char*>(workspace) + kHeader);
-  int e = map_cuda(launch_dvl(scores, B, L, budget, verify_len, offsets, slot_map, status, ticket, st));
+  int e = map_cuda(launch_dvl(scores, B, L, budget, verify_len, offsets, slot_map, status, st));
   if (e || !pack) return e;
   return map_cuda(launch_pack(dense_target, packed_target, dtype, B, L, V, budget, offsets, st));
 }

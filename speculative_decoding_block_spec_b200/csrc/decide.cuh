@@ -234,6 +234,119 @@ __device__ __forceinline__ DecideOut decide_warp_fp64(const DecideIn& in, const 
   return o;
 }
 
+// ------------------------------------------------- top-p filtered decisions
+
+// Inputs of one request's decision when every row is filtered to its top-p
+// nucleus ("DBLAST", Pith review, "What would settle it" and "Assumptions":
+// target probabilities under the same sampling filter). Row layout as in
+// DecideIn. The filtered log-probability of the drafted token in row q is
+// (xg - m) / T - lf when the token is in the row's nucleus (in[q] != 0),
+// else -inf; lf is the log of the row's nucleus mass sum 2^((x - m) k).
+struct DecideTopP {
+  const float* xg;
+  const float* m;
+  const double* lf;
+  const unsigned char* in;
+  const double* lw;  // log q(z|y) [K], nullptr for w = 1 (K == 1)
+  int ell, K, L;
+  float T;
+};
+
+// log sum exp over the first K entries; -inf when every entry is -inf.
+__device__ __forceinline__ double lse_k(const double* a, int K) {
+  double m = -INFINITY;
+#pragma unroll
+  for (int z = 0; z < kMaxK; ++z)
+    if (z < K) m = fmax(m, a[z]);
+  if (m == -INFINITY) return -INFINITY;
+  double s = 0.0;
+#pragma unroll
+  for (int z = 0; z < kMaxK; ++z)
+    if (z < K) s += exp(a[z] - m);
+  return m + log(s);
+}
+
+// Run by the 32 lanes of one warp (lane i tests position i), in fp64 with
+// the filtered rows. A token outside the target's nucleus has p = 0 and is
+// rejected (rho = 0); a token the filtered proposal gives 0 has rho = +inf
+// and is accepted; a posterior whose normaliser is not finite (every
+// category gives an accepted token probability 0) marks the request bad.
+__device__ __forceinline__ DecideOut decide_warp_topp(const DecideTopP& in, const float* u) {
+  const int lane = threadIdx.x & 31;
+  const int ell = in.ell, K = in.K;
+  const double T = static_cast<double>(in.T);
+  const bool act = lane < ell;
+  double lp = 0.0, lqz[kMaxK];
+#pragma unroll
+  for (int z = 0; z < kMaxK; ++z) lqz[z] = 0.0;
+  if (act) {
+    lp = in.in[lane] ? (static_cast<double>(in.xg[lane]) - static_cast<double>(in.m[lane])) / T - in.lf[lane]
+                     : -INFINITY;
+#pragma unroll
+    for (int z = 0; z < kMaxK; ++z) {
+      if (z < K) {
+        const int q = ell + z * ell + lane;
+        lqz[z] = in.in[q] ? (static_cast<double>(in.xg[q]) - static_cast<double>(in.m[q])) / T - in.lf[q]
+                          : -INFINITY;
+      }
+    }
+  }
+  // log pi_i(z) = log w_z + sum_{k<i} log q_k(x_k|y,z) - logsumexp_z(.)
+  double lpi[kMaxK];
+#pragma unroll
+  for (int z = 0; z < kMaxK; ++z) {
+    lpi[z] = -INFINITY;
+    if (z < K) {
+      double v = __shfl_up_sync(0xffffffffu, lqz[z], 1);
+      if (lane == 0) v = 0.0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const double t = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += t;
+      }
+      lpi[z] = (in.lw ? in.lw[z] : 0.0) + v;
+    }
+  }
+  const double norm = lse_k(lpi, K);
+  const bool bad = !isfinite(norm);
+  double t[kMaxK];
+#pragma unroll
+  for (int z = 0; z < kMaxK; ++z) {
+    lpi[z] = bad ? -INFINITY : lpi[z] - norm;
+    t[z] = lpi[z] + lqz[z];
+  }
+  const double lq = lse_k(t, K);
+  const double rho = lp == -INFINITY ? 0.0 : exp(lp - lq);
+  const double thr = fmin(1.0, rho);
+  const float uu = act ? u[lane] : 0.f;
+  const bool acc = static_cast<double>(uu) < thr;
+  const unsigned stop = __ballot_sync(0xffffffffu, act && (bad || isnan(rho) || !acc));
+  DecideOut o;
+  o.j = stop ? __ffs(stop) - 1 : ell;
+  o.bad = (__shfl_sync(0xffffffffu, (bad || isnan(rho)) ? 1 : 0, o.j & 31) && stop) ? 1 : 0;
+  o.ct = o.mt = 0.f;
+  const int src = o.j & 31;
+  double lpj[kMaxK];
+#pragma unroll
+  for (int z = 0; z < kMaxK; ++z) lpj[z] = __shfl_sync(0xffffffffu, lpi[z], src);
+  if (o.j < ell) {  // terminal multipliers of the residual at j: p = 2^((x - mt) k) ct, q = sum_z 2^((x - mz) k) cz
+    o.ct = static_cast<float>(exp(-in.lf[o.j]));
+    o.mt = in.m[o.j];
+#pragma unroll
+    for (int z = 0; z < kMaxK; ++z) {
+      if (z < K) {
+        const int q = ell + z * ell + o.j;
+        o.cz[z] = static_cast<float>(exp(lpj[z] - in.lf[q]));
+        o.mz[z] = in.m[q];
+      } else {
+        o.cz[z] = 0.f;
+        o.mz[z] = 0.f;
+      }
+    }
+  }
+  return o;
+}
+
 // ------------------------------------------------------------ terminal draw
 
 struct Best {

@@ -10,12 +10,22 @@
 // to the largest P overall, ordered (P desc, b asc, i asc); because each
 // row's products are non-increasing the chosen set is a prefix of every row.
 //
-// k_dvl_allocate: one block per request. Every block forms all B*L products
-// in shared memory (fp64, left to right), ranks its own L entries against
-// all of them, and writes verify_len[b]. The last block (atomic ticket,
-// reset by that block) scans the lengths into offsets and fills the slot
-// map. k_dvl_pack then copies the selected dense target rows into the
-// fixed-address packed buffer.
+// k_dvl_allocate: one block of 1024 threads does the whole allocation, in
+// shared memory, with no cross-block hand-off:
+//  1. one thread per request forms its products in fp64, left to right, and
+//     stores them as 64-bit keys whose unsigned order is the order of P
+//     (+0 and -0 are one key, as they compare equal);
+//  2. a radix select over the keys, eight 8-bit digits from the top, finds
+//     the key K of the (budget' - B)-th entry in the order (P desc, flat
+//     index asc): per digit a 256-bin histogram of the entries that still
+//     match the prefix, and one warp's suffix scan over it;
+//  3. entries with key > K are selected, and of those equal to K the first
+//     ones by flat index (an exclusive scan over the equal-key flags, only
+//     when some entries share K and not all of them are taken);
+//  4. verify_len[b] = selected entries of row b; an exclusive scan of
+//     verify_len + 1 gives the offsets, from which the slot map is filled.
+// O(B L) work per digit; k_dvl_pack then copies the selected dense target
+// rows into the fixed-address packed buffer.
 #include <algorithm>
 
 #include "common.cuh"
@@ -23,89 +33,142 @@
 
 namespace specv {
 
-constexpr int kDvlMaxL = 32;
+constexpr int kDvlThreads = 1024;
+constexpr int kDvlWarps = kDvlThreads / 32;
 
-__global__ void __launch_bounds__(kThreads) k_dvl_allocate(const float* __restrict__ scores, int B, int L,
-                                                           int budget, int32_t* verify_len, int32_t* offsets,
-                                                           int32_t* slot_map, int* status, int* ticket) {
-  extern __shared__ double sP[];  // [B*L] products; reused as int[B+1] by the last block
-  __shared__ int s_cnt[kDvlMaxL][kWarps];
-  __shared__ int s_tmp[kWarps + 1];
-  __shared__ int s_last;
+// Order-preserving key of a product: unsigned order of the key = numeric
+// order of P (negative values below +0; -0 maps to the key of +0; a NaN,
+// possible only from a flagged score, lands at one end).
+__device__ __forceinline__ unsigned long long p_key(double P) {
+  if (P == 0.0) P = 0.0;
+  const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(P));
+  return (b >> 63) ? ~b : (b | (1ull << 63));
+}
+
+__global__ void __launch_bounds__(kDvlThreads, 1) k_dvl_allocate(const float* __restrict__ scores, int B, int L,
+                                                               int budget, int32_t* verify_len, int32_t* offsets,
+                                                               int32_t* slot_map, int* status) {
+  extern __shared__ unsigned long long sKey[];  // [B*L] keys, then int[B*L] equal-key ranks, int[B + 1] lengths
+  __shared__ int s_hist[256];
+  __shared__ int s_tmp[kDvlWarps + 1];
+  __shared__ int s_digit, s_k, s_eq, s_flag;
   pdl_wait();
   pdl_trigger();
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  const int b = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int n = B * L;
+  int* sRank = reinterpret_cast<int*>(sKey + n);  // index-order rank among the entries equal to the cut key
+  int* lens = sRank + n;                           // verify_len + 1, then offsets
 
-  for (int r = tid; r < B; r += kThreads) {
+  if (tid == 0) {
+    s_flag = 0;
+    s_eq = 0;
+  }
+  __syncthreads();
+  int bad = 0;
+  for (int r = tid; r < B; r += kDvlThreads) {
     double P = 1.0;
     for (int i = 0; i < L; ++i) {
-      P = P * static_cast<double>(scores[static_cast<int64_t>(r) * L + i]);
-      sP[r * L + i] = P;
+      const float s = scores[static_cast<int64_t>(r) * L + i];
+      bad |= !(s >= 0.f && s <= 1.f);
+      P = P * static_cast<double>(s);
+      sKey[r * L + i] = p_key(P);
     }
   }
-  if (tid < L) {
-    const float s = scores[static_cast<int64_t>(b) * L + tid];
-    if (!(s >= 0.f && s <= 1.f)) atomicOr(status, kFlagScores);
-  }
-  __syncthreads();
+  if (bad) atomicOr(&s_flag, kFlagScores);
 
   const int64_t cap = static_cast<int64_t>(B) * (L + 1);
-  const int take = static_cast<int>(std::min<int64_t>(budget, cap)) - B;
-  // rank of (b, i) = number of entries ordered before it
-  for (int i = 0; i < L; ++i) {
-    const double Pi = sP[b * L + i];
-    const int self = b * L + i;
-    int c = 0;
-    for (int e = tid; e < n; e += kThreads) {
-      const double Pe = sP[e];
-      c += (Pe > Pi || (Pe == Pi && e < self)) ? 1 : 0;
-    }
+  const int take = static_cast<int>(std::min<int64_t>(budget, cap)) - B;  // 0 <= take <= n
+  unsigned long long kth = ~0ull;  // take == 0: nothing is selected (no key exceeds ~0)
+  int k_eq = 0;                    // entries equal to kth that are taken
+  if (take > 0) {
+    unsigned long long prefix = 0, mask = 0;
+    int k = take;  // rank (1-based, descending) of the wanted entry among those matching the prefix
+    for (int shift = 56; shift >= 0; shift -= 8) {
+      if (tid < 256) s_hist[tid] = 0;
+      __syncthreads();
+      for (int e = tid; e < n; e += kDvlThreads) {
+        const unsigned long long u = sKey[e];
+        if ((u & mask) == prefix) atomicAdd(&s_hist[(u >> shift) & 255], 1);
+      }
+      __syncthreads();
+      if (wid == 0) {  // lane l owns digits 255 - 8l ... 248 - 8l (descending)
+        int c[8], sum = 0;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-    if (lane == 0) s_cnt[i][w] = c;
+        for (int t = 0; t < 8; ++t) {
+          c[t] = s_hist[255 - 8 * lane - t];
+          sum += c[t];
+        }
+        int incl = sum;  // inclusive scan over lanes: entries in digits above and including this lane's
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        const int excl = incl - sum;
+        if (excl < k && incl >= k) {  // the wanted entry's digit is in this lane's range
+          int run = excl;
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            if (run < k && run + c[t] >= k) {
+              s_digit = 255 - 8 * lane - t;
+              s_k = k - run;
+            }
+            run += c[t];
+          }
+        }
+      }
+      __syncthreads();
+      // s_digit and s_k are rewritten only after two more barriers of the next digit
+      prefix |= static_cast<unsigned long long>(s_digit) << shift;
+      mask |= 255ull << shift;
+      k = s_k;
+    }
+    kth = prefix;
+    k_eq = k;
   }
-  __syncthreads();
-  if (tid < L) {
-    int rank = 0;
-    for (int k = 0; k < kWarps; ++k) rank += s_cnt[tid][k];
-    s_cnt[tid][0] = rank < take ? 1 : 0;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    int ell = 0;
-    for (int i = 0; i < L; ++i) ell += s_cnt[i][0];
-    verify_len[b] = ell;
-    __threadfence();
-    s_last = atomicAdd(ticket, 1) == B - 1;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
 
-  int* off = reinterpret_cast<int*>(sP);
-  for (int r = tid; r < B; r += kThreads) off[r] = __ldcg(verify_len + r) + 1;
+  // entries equal to kth: the first k_eq of them by flat index are taken
+  int n_eq_local = 0;
+  for (int e = tid; e < n; e += kDvlThreads) n_eq_local += sKey[e] == kth;
+  if (n_eq_local) atomicAdd(&s_eq, n_eq_local);
   __syncthreads();
-  const int total = block_exclusive_scan(off, B, s_tmp);
-  if (tid == 0) off[B] = total;
+  const bool rank_eq = s_eq > k_eq && k_eq > 0;  // only then does the index order among equals matter
+  if (rank_eq) {
+    for (int e = tid; e < n; e += kDvlThreads) sRank[e] = sKey[e] == kth;
+    __syncthreads();
+    block_exclusive_scan<kDvlThreads>(sRank, n, s_tmp);
+  }
+  // verify_len[b]: selected entries of row b (a prefix of the row when every score is in [0, 1])
+  for (int r = tid; r < B; r += kDvlThreads) {
+    int ell = 0;
+    for (int i = 0; i < L; ++i) {
+      const int e = r * L + i;
+      const unsigned long long u = sKey[e];
+      ell += (u > kth || (u == kth && (rank_eq ? sRank[e] < k_eq : k_eq > 0))) ? 1 : 0;
+    }
+    verify_len[r] = ell;
+    lens[r] = ell + 1;
+  }
   __syncthreads();
-  for (int r = tid; r <= B; r += kThreads) offsets[r] = off[r];
+  const int total = block_exclusive_scan<kDvlThreads>(lens, B, s_tmp);
+  if (tid == 0) lens[B] = total;
+  __syncthreads();
+  for (int r = tid; r <= B; r += kDvlThreads) offsets[r] = lens[r];
   if (slot_map) {
-    for (int s = tid; s < budget; s += kThreads) {
+    for (int s = tid; s < budget; s += kDvlThreads) {
       int v = -1;
       if (s < total) {
-        int lo = 0, hi = B - 1;  // last request with off <= s
+        int lo = 0, hi = B - 1;  // last request with offset <= s
         while (lo < hi) {
           const int mid = (lo + hi + 1) >> 1;
-          if (off[mid] <= s) lo = mid; else hi = mid - 1;
+          if (lens[mid] <= s) lo = mid; else hi = mid - 1;
         }
-        v = lo * (L + 1) + (s - off[lo]);
+        v = lo * (L + 1) + (s - lens[lo]);
       }
       slot_map[s] = v;
     }
   }
-  if (tid == 0) *ticket = 0;
+  if (tid == 0 && s_flag) atomicOr(status, s_flag);
 }
 
 // packed[offsets[b] + i] = dense[b, i] for i <= verify_len[b]; one block per
@@ -145,15 +208,17 @@ __global__ void __launch_bounds__(kThreads) k_dvl_pack(const char* __restrict__ 
 }
 
 cudaError_t launch_dvl(const float* scores, int B, int L, int budget, int32_t* verify_len, int32_t* offsets,
-                       int32_t* slot_map, int* status, int* ticket, cudaStream_t st) {
-  const size_t smem = std::max(static_cast<size_t>(B) * L * sizeof(double), static_cast<size_t>(B + 1) * sizeof(int));
+                       int32_t* slot_map, int* status, cudaStream_t st) {
+  const int64_t n = static_cast<int64_t>(B) * L;
+  const size_t smem = static_cast<size_t>(n) * (sizeof(unsigned long long) + sizeof(int)) +
+                      static_cast<size_t>(B + 1) * sizeof(int);
   if (smem > 48 * 1024) {
     const cudaError_t e =
         cudaFuncSetAttribute(k_dvl_allocate, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  return launch_pdl(k_dvl_allocate, dim3(B), dim3(kThreads), smem, st, scores, B, L, budget, verify_len, offsets,
-                    slot_map, status, ticket);
+  return launch_pdl(k_dvl_allocate, dim3(1), dim3(kDvlThreads), smem, st, scores, B, L, budget, verify_len, offsets,
+                    slot_map, status);
 }
 
 cudaError_t launch_pack(const void* dense, void* packed, int dtype, int B, int L, int64_t V, int budget,

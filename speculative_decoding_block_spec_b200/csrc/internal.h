@@ -8,10 +8,11 @@ namespace specv {
 
 // The rows walked by the row-statistics kernel.
 //  plain  (verify == 0): row r at target + r * stride elements, r < rows.
-//  verify (verify == 1): request b contributes (K+1) * l_b rows, l_b =
-//    verify_len[b] (L if NULL): first target rows 0..l_b-1 (row of (b, i) is
-//    row_off[b] + i, or b*(L+1) + i when row_off is NULL), then draft rows
-//    (z, i) for z < K, i < l_b at draft + ((b*K + z)*L + i) * V.
+//  verify (verify == 1): request b contributes (K+1) * l_b + bonus rows, l_b =
+//    verify_len[b] (L if NULL): first target rows 0..l_b-1, and row l_b too
+//    when bonus == 1 (row of (b, i) is row_off[b] + i, or b*(L+1) + i when
+//    row_off is NULL), then draft rows (z, i) for z < K, i < l_b at
+//    draft + ((b*K + z)*L + i) * V.
 struct RowSpace {
   const void* target;
   const void* draft;
@@ -23,6 +24,7 @@ struct RowSpace {
   int64_t rows;
   int B, L, K;
   int verify;
+  int bonus;                // verify mode: 1 to include each request's bonus row (top-p filtering)
 };
 
 // Everything the accept/sample kernel reads and writes.
@@ -48,6 +50,26 @@ struct VerifyArgs {
   int G;                    // row-statistics grid size
   int64_t Vu;               // row-statistics units per row
   int P;                    // sampling blocks per request
+  int topp;                 // rows filtered to their top-p nuclei: the fields below replace xg's partials
+  const float* nuc_m;       // [walk rows] row maxima (walk with bonus rows)
+  const double* nuc_lf;     // [walk rows] log nucleus masses
+  const uint32_t* nuc_key;  // [walk rows] cut keys
+  const int32_t* nuc_v;     // [walk rows] cut tokens
+};
+
+// The top-p nucleus kernel's inputs and outputs (one entry per walk row).
+struct NucleusArgs {
+  RowSpace rs;              // the verify walk, bonus rows included
+  const float2* part;       // row-statistics partials of that walk
+  int G;                    // row-statistics grid size
+  int64_t Vu;               // row-statistics units per row
+  int64_t V;
+  float k;                  // log2(e) / T
+  double top_p;
+  float* row_m;             // out: row maximum (raw logit), NaN for a non-finite row
+  double* row_lf;           // out: log of the nucleus mass sum_{v kept} 2^((x_v - m) k)
+  uint32_t* cut_key;        // out: order key of the cut value
+  int32_t* cut_v;           // out: cut token (tokens at the cut value with index <= cut_v are kept)
 };
 
 // Units of work per row: 16-byte vectors on the vector path, else elements.
@@ -65,12 +87,13 @@ cudaError_t launch_softmax_finalize(const void* logits, int dtype, bool vec, int
                                     int64_t stride, float T, int G, const float2* part, float* row_max,
                                     float* row_lse, float* probs, cudaStream_t st);
 
+cudaError_t launch_nucleus(const NucleusArgs& a, int dtype, bool vec, cudaStream_t st);
+
 cudaError_t launch_accept_sample(const VerifyArgs& a, int dtype, bool vec, cudaStream_t st);
-int accept_blocks_per_sm(int dtype, bool vec, int K);
+int accept_blocks_per_sm(int dtype, bool vec, int K, bool topp);
 
 cudaError_t launch_dvl(const float* scores, int B, int L, int budget, int32_t* verify_len,
-                       int32_t* offsets, int32_t* slot_map, int* status, int* ticket,
-                       cudaStream_t st);
+                       int32_t* offsets, int32_t* slot_map, int* status, cudaStream_t st);
 
 cudaError_t launch_pack(const void* dense, void* packed, int dtype, int B, int L, int64_t V,
                         int budget, const int32_t* offsets, cudaStream_t st);

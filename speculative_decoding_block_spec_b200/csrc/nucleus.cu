@@ -1,0 +1,340 @@
+// Top-p (nucleus) cut of every row of the verify window.
+//
+// Target sampling with a temperature and a top-p filter, target
+// probabilities taken under the same sampling filter ("DBLAST: Dependent
+// Block Drafting for Stochastic Speculative Decoding", Pith review, "What
+// would settle it": T = 1.5, top-p 0.95; "Assumptions"). The filter of a row
+// keeps its nucleus: the shortest run of tokens, in the order (probability
+// descending, index ascending), whose mass reaches top_p; the kept tokens
+// are renormalised and every other token gets probability 0. The same filter
+// applies to the target rows and to every draft category.
+//
+// Probability is monotone in the logit, so the order is that of the logits,
+// and the nucleus is fixed by a cut: the logit value x_c and token v_c of its
+// last member; token v is kept iff x_v > x_c, or x_v == x_c and v <= v_c.
+//
+// k_nucleus, one row at a time per block (rows strided over the grid):
+//  1. the row's maximum m from the statistics partials;
+//  2. a radix descent over 32-bit order keys of the logits (bf16 logits
+//     widened exactly to fp32): per digit, a shared-memory histogram of the
+//     mass of the tokens that match the key prefix found so far, then a
+//     descending scan for the digit whose bin carries the running mass
+//     across top_p * total. Digits: bits 31..20 (4096 bins), then 19..16 for
+//     bf16 (whose low 16 bits are fixed by the sign), or 19..8 and 7..0 for
+//     fp32. Masses are 2^((x - m) k) in fixed point (scaled by 2^42, rounded
+//     to the nearest unit) summed with 64-bit integer atomics, so every sum
+//     is exact and independent of the order the atomics land in;
+//  3. at the cut value, the number n of its tokens needed to reach top_p;
+//     if not all of them are needed, the n-th such token in index order is
+//     found with a warp-ordered count (the tie cut);
+//  4. outputs: m, the log of the nucleus mass sum_{v kept} 2^((x_v - m) k)
+//     (the filtered rows' normaliser), the cut key and the cut token.
+// The first digit streams the row from HBM; the later passes find it in L2.
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+#include "walk.cuh"
+
+namespace specv {
+
+constexpr int kNucThreads = 512;
+constexpr int kNucWarps = kNucThreads / 32;
+constexpr int kFix = 42;              // fixed-point scale of the masses: sums of up to 2^20 terms of <= 1 fit 2^62
+constexpr int kNucBins = 4096;        // bins of the widest digit
+constexpr int kNucCountBins = 256;    // bins of the last digit, which also counts tokens
+
+// round(q * 2^kFix) for q in [0, 1] (fp32 bits; no conversion instruction).
+__device__ __forceinline__ unsigned long long to_fixed(float q) {
+  const uint32_t b = __float_as_uint(q);
+  const int e = static_cast<int>(b >> 23);
+  if (e == 0) return 0ull;
+  const uint32_t mant = (b & 0x7FFFFFu) | 0x800000u;  // q = mant * 2^(e - 150)
+  const int sh = e - 150 + kFix;
+  if (sh >= 0) return static_cast<unsigned long long>(mant) << sh;
+  if (sh <= -25) return 0ull;                          // below half a unit
+  return static_cast<unsigned long long>((mant + (1u << (-sh - 1))) >> (-sh));
+}
+
+// Block-wide exclusive scan of one 64-bit value per thread (thread order);
+// `tmp` holds kNucWarps + 1 values. Returns the exclusive prefix.
+__device__ __forceinline__ unsigned long long block_scan_u64(unsigned long long v, unsigned long long* tmp) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  unsigned long long incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) tmp[w] = incl;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long run = 0;
+    for (int k = 0; k < kNucWarps; ++k) {
+      const unsigned long long t = tmp[k];
+      tmp[k] = run;
+      run += t;
+    }
+    tmp[kNucWarps] = run;
+  }
+  __syncthreads();
+  const unsigned long long excl = tmp[w] + incl - v;
+  __syncthreads();
+  return excl;
+}
+
+// One digit of the descent: hist[d] += fixed mass of every token whose key
+// matches `prefix` under `pmask`, d = (key >> shift) & dmask; with `count`
+// also cnt[d] += 1. Called by the whole block.
+template <int DT, bool VEC>
+__device__ __forceinline__ void digit_pass(const char* row, int64_t V, float m, float k, uint32_t prefix,
+                                           uint32_t pmask, int shift, uint32_t dmask, bool count,
+                                           unsigned long long* hist, unsigned* cnt) {
+  constexpr int E = VEC ? Elem<DT>::kPerVec : 1;
+  constexpr int U = VEC ? 2 : 1;  // units in flight per thread
+  const int64_t Vu = V / E;
+  for (int64_t u0 = threadIdx.x; u0 < Vu; u0 += U * kNucThreads) {
+    float x[U][E];
+#pragma unroll
+    for (int h = 0; h < U; ++h) {
+      const int64_t u = u0 + static_cast<int64_t>(h) * kNucThreads;
+      if (u >= Vu) break;
+      if constexpr (VEC) Elem<DT>::unpack(ldg16(reinterpret_cast<const uint4*>(row) + u), x[h]);
+      else x[h][0] = Elem<DT>::at(row, u);
+    }
+#pragma unroll
+    for (int h = 0; h < U; ++h) {
+      if (u0 + static_cast<int64_t>(h) * kNucThreads >= Vu) break;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const uint32_t key = order_key(x[h][e]);
+        if ((key & pmask) != prefix) continue;
+        const uint32_t d = (key >> shift) & dmask;
+        const unsigned long long fx = to_fixed(ex2((x[h][e] - m) * k));
+        if (fx) atomicAdd(&hist[d], fx);
+        if (count) atomicAdd(&cnt[d], 1u);
+      }
+    }
+  }
+}
+
+// The digit d, scanning bins nb-1 down to 0 from the running mass `above`,
+// whose bin takes the running mass from below `target` to at least it; also
+// the running mass above that bin. Called by the whole block.
+__device__ __forceinline__ void find_digit(const unsigned long long* hist, int nb, unsigned long long above,
+                                           unsigned long long target, unsigned long long* tmp, int* s_d,
+                                           unsigned long long* s_above) {
+  if (threadIdx.x == 0) {  // defaults, overwritten by the one thread whose bins hold the crossing
+    *s_d = 0;
+    *s_above = above;
+  }
+  const int per = (nb + kNucThreads - 1) / kNucThreads;
+  const int hi = nb - 1 - threadIdx.x * per;  // this thread's bins: hi, hi - 1, ... (descending)
+  unsigned long long local = 0;
+  for (int t = 0; t < per; ++t)
+    if (hi - t >= 0) local += hist[hi - t];
+  unsigned long long run = above + block_scan_u64(local, tmp);
+  for (int t = 0; t < per; ++t) {
+    const int d = hi - t;
+    if (d < 0) break;
+    const unsigned long long h = hist[d];
+    if (run < target && run + h >= target) {
+      *s_d = d;
+      *s_above = run;
+    }
+    run += h;
+  }
+  __syncthreads();
+}
+
+// Index (in row order) of the n-th token (1-based) whose key is kappa; the
+// row holds at least n of them. Called by the whole block.
+template <int DT, bool VEC>
+__device__ __forceinline__ int64_t nth_equal(const char* row, int64_t V, uint32_t kappa, unsigned n, unsigned* s_wc,
+                                             long long* s_v) {
+  constexpr int E = VEC ? Elem<DT>::kPerVec : 1;
+  const int64_t Vu = V / E;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t cw = (Vu + kNucWarps - 1) / kNucWarps;  // units per warp, contiguous
+  const int64_t a = min(Vu, w * cw), b = min(Vu, a + cw);
+  auto matches = [&](int64_t u) -> unsigned {  // bit e set when element e of unit u has key kappa
+    float x[E];
+    if constexpr (VEC) Elem<DT>::unpack(ldg16(reinterpret_cast<const uint4*>(row) + u), x);
+    else x[0] = Elem<DT>::at(row, u);
+    unsigned bits = 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) bits |= (order_key(x[e]) == kappa ? 1u : 0u) << e;
+    return bits;
+  };
+  if (threadIdx.x == 0) *s_v = V - 1;  // overwritten by the lane that finds the token
+  unsigned c = 0;
+  for (int64_t u = a + lane; u < b; u += 32) c += __popc(matches(u));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if (lane == 0) s_wc[w] = c;
+  __syncthreads();
+  unsigned base = 0;
+  for (int k = 0; k < w; ++k) base += s_wc[k];
+  if (base < n && base + s_wc[w] >= n) {  // this warp holds the n-th: walk its units in order
+    unsigned run = base;
+    for (int64_t u0 = a; u0 < b; u0 += 32) {
+      const int64_t u = u0 + lane;
+      const unsigned bits = u < b ? matches(u) : 0u;
+      unsigned incl = __popc(bits);
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      const unsigned before = run + incl - __popc(bits);
+      if (before < n && run + incl >= n) {  // in this lane's unit: the (n - before)-th set bit
+        unsigned need = n - before, bb = bits;
+        for (int e = 0; e < E; ++e) {
+          if (bb & 1u) {
+            if (--need == 0) {
+              *s_v = u * E + e;
+              break;
+            }
+          }
+          bb >>= 1;
+        }
+      }
+      run += __shfl_sync(0xffffffffu, incl, 31);
+      if (run >= n) break;
+    }
+  }
+  __syncthreads();
+  return *s_v;
+}
+
+template <int DT, bool VEC>
+__global__ void __launch_bounds__(kNucThreads, 2) k_nucleus(NucleusArgs a) {
+  extern __shared__ unsigned long long nuc_smem[];  // hist[kNucBins], then walk rowoff[B + 1], base[B]
+  unsigned long long* hist = nuc_smem;
+  int* walk_smem = reinterpret_cast<int*>(nuc_smem + kNucBins);
+  __shared__ unsigned s_cnt[kNucCountBins];
+  __shared__ unsigned long long s_tmp[kNucWarps + 1];
+  __shared__ int s_itmp[kNucWarps + 1];
+  __shared__ unsigned s_wc[kNucWarps];
+  __shared__ float s_m;
+  __shared__ const char* s_row;
+  __shared__ int s_d;
+  __shared__ unsigned long long s_above;
+  __shared__ long long s_v;
+  pdl_wait();
+  pdl_trigger();
+  const RowSpace& rs = a.rs;
+  const Walk w{walk_smem, walk_smem + rs.B + 1};
+  const int64_t nrows = build_walk<kNucThreads>(rs, walk_smem, s_itmp);
+  const int64_t N = nrows * a.Vu;
+  const int tid = threadIdx.x;
+  const bool bf16 = DT == 1;
+  for (int64_t r = blockIdx.x; r < nrows; r += gridDim.x) {
+    if (tid == 0) {
+      float m, s;
+      merge_row(a.part, r, a.Vu, N, a.G, a.k, m, s);
+      s_m = (isfinite(m) && isfinite(s)) ? m : NAN;
+      const int32_t* tokp;
+      s_row = locate<DT>(rs, w, r, tokp);
+    }
+    for (int i = tid; i < kNucBins; i += kNucThreads) hist[i] = 0ull;
+    for (int i = tid; i < kNucCountBins; i += kNucThreads) s_cnt[i] = 0u;
+    __syncthreads();
+    const float m = s_m;
+    const char* row = s_row;
+    if (!(m == m)) {  // a non-finite row: the sampling kernel flags the request
+      if (tid == 0) {
+        a.row_m[r] = NAN;
+        a.row_lf[r] = NAN;
+        a.cut_key[r] = 0u;
+        a.cut_v[r] = static_cast<int32_t>(a.V - 1);
+      }
+      __syncthreads();
+      continue;
+    }
+    // digit 1: bits 31..20, every token; its total is the row's whole mass
+    digit_pass<DT, VEC>(row, a.V, m, a.k, 0u, 0u, 20, 0xFFFu, false, hist, s_cnt);
+    __syncthreads();
+    unsigned long long local = 0;
+    for (int i = tid; i < kNucBins; i += kNucThreads) local += hist[i];
+    const unsigned long long total = block_scan_u64(local, s_tmp) + local;  // the last thread's inclusive sum
+    if (tid == kNucThreads - 1) s_above = total;
+    __syncthreads();
+    const unsigned long long whole = s_above;
+    unsigned long long target = static_cast<unsigned long long>(ceil(a.top_p * static_cast<double>(whole)));
+    if (target < 1ull) target = 1ull;
+    if (target > whole) target = whole;
+    __syncthreads();
+    find_digit(hist, kNucBins, 0ull, target, s_tmp, &s_d, &s_above);
+    uint32_t prefix = static_cast<uint32_t>(s_d) << 20, pmask = 0xFFF00000u;
+    unsigned long long above = s_above;
+    int nb, shift;
+    if (bf16) {  // digit 2: bits 19..16, which complete a widened bf16 key
+      shift = 16;
+      nb = 16;
+    } else {     // digit 2: bits 19..8
+      shift = 8;
+      nb = kNucBins;
+    }
+    __syncthreads();
+    for (int i = tid; i < kNucBins; i += kNucThreads) hist[i] = 0ull;
+    __syncthreads();
+    digit_pass<DT, VEC>(row, a.V, m, a.k, prefix, pmask, shift, static_cast<uint32_t>(nb - 1), bf16, hist, s_cnt);
+    __syncthreads();
+    find_digit(hist, nb, above, target, s_tmp, &s_d, &s_above);
+    int dl = s_d;
+    prefix |= static_cast<uint32_t>(dl) << shift;
+    above = s_above;
+    uint32_t kappa;
+    if (bf16) {
+      kappa = prefix | ((prefix & 0x80000000u) ? 0u : 0xFFFFu);  // the low half of a widened bf16 key
+    } else {     // digit 3: bits 7..0, with token counts
+      pmask = 0xFFFFFF00u;
+      __syncthreads();
+      for (int i = tid; i < kNucCountBins; i += kNucThreads) hist[i] = 0ull;
+      __syncthreads();
+      digit_pass<DT, VEC>(row, a.V, m, a.k, prefix, pmask, 0, 0xFFu, true, hist, s_cnt);
+      __syncthreads();
+      find_digit(hist, kNucCountBins, above, target, s_tmp, &s_d, &s_above);
+      dl = s_d;
+      above = s_above;
+      kappa = prefix | static_cast<uint32_t>(dl);
+    }
+    // tokens at the cut value: how many are needed, and which is the last
+    const unsigned c = s_cnt[dl];
+    const unsigned long long each = hist[dl] / c;  // every token of the cut value has the same mass
+    const unsigned long long need = (target - above + each - 1) / each;
+    const unsigned take = static_cast<unsigned>(need < c ? need : c);
+    const unsigned long long kept = above + static_cast<unsigned long long>(take) * each;
+    __syncthreads();
+    int64_t vcut = a.V - 1;
+    if (take < c) vcut = nth_equal<DT, VEC>(row, a.V, kappa, take, s_wc, &s_v);
+    if (tid == 0) {
+      a.row_m[r] = m;
+      a.row_lf[r] = log(static_cast<double>(kept)) - kFix * 0.6931471805599453;
+      a.cut_key[r] = kappa;
+      a.cut_v[r] = static_cast<int32_t>(vcut);
+    }
+    __syncthreads();
+  }
+}
+
+cudaError_t launch_nucleus(const NucleusArgs& a, int dtype, bool vec, cudaStream_t st) {
+  const size_t smem = kNucBins * sizeof(unsigned long long) + static_cast<size_t>(2 * a.rs.B + 1) * sizeof(int);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t rows_max = static_cast<int64_t>(a.rs.B) * ((a.rs.K + 1) * a.rs.L + 1);
+  const dim3 grid(static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(rows_max, 3 * sms))));
+  auto go = [&](auto kernel) {
+    if (smem > 48 * 1024) {
+      const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+    }
+    return launch_pdl(kernel, grid, dim3(kNucThreads), smem, st, a);
+  };
+  if (dtype == 0) return vec ? go(k_nucleus<0, true>) : go(k_nucleus<0, false>);
+  return vec ? go(k_nucleus<1, true>) : go(k_nucleus<1, false>);
+}
+
+}  // namespace specv

@@ -22,46 +22,11 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "walk.cuh"
 
 namespace specv {
 
 constexpr int kUnroll = 4;  // 16-byte vectors in flight per thread per group
-
-// Geometry of the verify walk, built in shared memory by every block:
-// rowoff[b] first walk row of request b (rowoff[B] = total), base[b] target
-// row of its position 0. Request b owns (K+1)*l walk rows: l target rows,
-// then K draft categories of l rows each, l = verified length.
-struct Walk {
-  const int* rowoff;
-  const int* base;
-};
-
-// Row r of the walk and the address of the drafted token of its position
-// (nullptr outside verify mode). The token itself is loaded by the caller,
-// which uses it only after the row's first data has arrived.
-template <int DT>
-__device__ __forceinline__ const char* locate(const RowSpace& rs, const Walk& w, int64_t r, const int32_t*& tokp) {
-  constexpr int64_t esz = Elem<DT>::kBytes;
-  tokp = nullptr;
-  if (!rs.verify) return static_cast<const char*>(rs.target) + r * rs.stride * esz;
-  int lo = 0, hi = rs.B - 1;  // last request whose first row is <= r
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (w.rowoff[mid] <= r) lo = mid; else hi = mid - 1;
-  }
-  const int b = lo;
-  const int q = static_cast<int>(r - w.rowoff[b]);
-  const int l = (w.rowoff[b + 1] - w.rowoff[b]) / (rs.K + 1);
-  if (q < l) {
-    tokp = rs.tokens + static_cast<int64_t>(b) * rs.L + q;
-    return static_cast<const char*>(rs.target) + (static_cast<int64_t>(w.base[b]) + q) * rs.stride * esz;
-  }
-  const int q2 = q - l, z = q2 / l, i = q2 - z * l;
-  tokp = rs.tokens + static_cast<int64_t>(b) * rs.L + i;
-  return static_cast<const char*>(rs.draft) + ((static_cast<int64_t>(b) * rs.K + z) * rs.L + i) * rs.stride * esz;
-}
-
-__device__ __forceinline__ int load_token(const int32_t* tokp) { return tokp ? __ldg(tokp) : -1; }
 
 // Vector path: each segment (the block's part of one row) streams groups of
 // kUnroll 16-byte vectors per thread, then single vectors, and ends with one
@@ -127,26 +92,6 @@ __device__ __forceinline__ void walk_scalar(const RowSpace& rs, const Walk& w, i
     if (threadIdx.x == 0) part[blockIdx.x + r] = make_float2(m, s);
     e = se;
   }
-}
-
-// Rows of the walk; in verify mode also builds its geometry in shared memory
-// (every thread of the block calls this).
-template <int NT>
-__device__ __forceinline__ int64_t build_walk(const RowSpace& rs, int* walk_smem, int* tmp) {
-  if (!rs.verify) return rs.rows;
-  int* rowoff = walk_smem;
-  int* base = walk_smem + rs.B + 1;
-  for (int b = threadIdx.x; b < rs.B; b += NT) {
-    int l = rs.vlen ? rs.vlen[b] : rs.L;
-    if (l < 0 || l > rs.L) l = 0;  // flagged by the sampling kernel
-    rowoff[b] = (rs.K + 1) * l;
-    base[b] = rs.row_off ? rs.row_off[b] : b * (rs.L + 1);
-  }
-  __syncthreads();
-  const int64_t nrows = block_exclusive_scan<NT>(rowoff, rs.B, tmp);
-  if (threadIdx.x == 0) rowoff[rs.B] = static_cast<int>(nrows);
-  __syncthreads();
-  return nrows;
 }
 
 template <int DT, bool VEC>
@@ -308,19 +253,6 @@ __global__ void __launch_bounds__(kDynThreads, 1) k_row_stats_dyn(RowSpace rs, i
   }
 }
 
-// Merge the partials of row r.
-__device__ __forceinline__ void merge_row(const float2* part, int64_t r, int64_t Vu, int64_t N, int G, float k,
-                                          float& m, float& s) {
-  const int64_t c0 = split_owner(r * Vu, N, G), c1 = split_owner((r + 1) * Vu - 1, N, G);
-  m = -INFINITY;
-  s = 0.f;
-  for (int64_t c = c0; c <= c1; ++c) {
-    if (split_start(c + 1, N, G) == split_start(c, N, G)) continue;  // empty share (N < grid): no partial
-    const float2 p = part[c + r];
-    ms_merge(m, s, p.x, p.y, k);
-  }
-}
-
 __global__ void __launch_bounds__(kThreads) k_softmax_stats(int64_t rows, int64_t Vu, int G, float k, float T,
                                                             const float2* __restrict__ part, float* row_max,
                                                             float* row_lse) {
@@ -438,7 +370,8 @@ cudaError_t launch_row_stats(const RowSpace& rs, int dtype, bool vec, int64_t V,
   const float k = log2e_over(T);
   const size_t smem = rs.verify ? static_cast<size_t>(2 * rs.B + 1) * sizeof(int) : 0;
   const dim3 grid(G), block(kThreads);
-  const int64_t max_units = (rs.verify ? static_cast<int64_t>(rs.B) * (rs.K + 1) * rs.L : rs.rows) * Vu;
+  const int64_t max_units =
+      (rs.verify ? static_cast<int64_t>(rs.B) * ((rs.K + 1) * rs.L + rs.bonus) : rs.rows) * Vu;
   if (use_dyn(vec, max_units, Vu, G))
     return dtype == 0 ? launch_pdl(k_row_stats_dyn<0>, grid, dim3(kDynThreads), smem, st, rs, Vu, G, k, part)
                       : launch_pdl(k_row_stats_dyn<1>, grid, dim3(kDynThreads), smem, st, rs, Vu, G, k, part);

@@ -4,8 +4,10 @@ compare the CUDA path's decisions with the oracle's under the low-margin rule.
 Rule: accepted lengths and tokens must match bit for bit. A decision whose
 oracle margin is below 1e-6 (accept test: |u - min(1, rho)|; terminal draw:
 the fp64 gap between the two best scores below 1e-6 * max(1, kappa), kappa =
-p / (p - q) being the amplification of rounding in log(p - q)) is logged in
-the run-wide tally. If the GPU differs from the oracle on such a request,
+p / (p - q) being the amplification of rounding in log(p - q); with top-p
+filtering, a nucleus boundary whose cumulative mass lies within 1e-6 of
+top-p, over the rows the request's outputs depend on) is logged in the
+run-wide tally. If the GPU differs from the oracle on such a request,
 the request is exempt from the comparison from that decision on (its earlier
 outputs must still match) and counts as an exempted difference. Over the
 whole test run the exempted differences must stay at or below 1e-5 of all
@@ -80,6 +82,13 @@ def check_verify(acc, out, ref, verify_len=None, log=None):
         low = [i for i in range(tested) if m[i] < EPS]
         n_dec += tested + 1
         same = acc[b] == ja and np.array_equal(out[b], ro)
+        nm = ref.get("nucleus_margin")
+        if nm is not None and nm[b] < EPS:  # top-p: a nucleus boundary the outputs depend on is low-margin
+            entry = (b, "nucleus", 0, float(nm[b]), bool(same))
+            low_here.append(entry)
+            if not same:
+                TALLY["exempted"].append(entry)
+            continue
         if low:
             i0 = low[0]
             entry = (b, "accept", i0, float(m[i0]), bool(same))

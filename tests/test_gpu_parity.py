@@ -409,7 +409,8 @@ def test_zero_length_block():
 # ---------------------------------------------------------------------- DVL
 
 @pytest.mark.parametrize("B,L,budget", [(1, 4, 1), (3, 4, 7), (32, 16, 272), (64, 16, 544), (16, 32, 300),
-                                        (7, 5, 100), (200, 16, 1700), (512, 32, 8000)])
+                                        (7, 5, 100), (200, 16, 1700), (512, 32, 8000), (4096, 4, 9000),
+                                        (9, 3, 9), (6, 4, 1000), (5, 0, 5), (4096, 1, 4097)])
 def test_dvl_parity(B, L, budget):
     rng = np.random.default_rng(B * 1000 + L)
     s = rng.beta(6.0, 2.0, size=(B, L)).astype(np.float32)
@@ -420,6 +421,30 @@ def test_dvl_parity(B, L, budget):
     np.testing.assert_array_equal(_cpu(vl), ref["verify_len"])
     np.testing.assert_array_equal(_cpu(off), ref["offsets"])
     np.testing.assert_array_equal(_cpu(sm), ref["slot_map"])
+
+
+@pytest.mark.parametrize("case", ["signed_zeros", "all_equal", "coarse_ties", "unsorted"])
+def test_dvl_ties_zeros_and_unsorted_rows(case):
+    """The order (P desc, b asc, i asc) decides every tie, -0 and +0 are
+    equal products, and rows whose scores are not sorted still get the
+    oracle's counts (the selection is then not a prefix of the row)."""
+    rng = np.random.default_rng(7)
+    B, L = 48, 12
+    if case == "signed_zeros":
+        s = rng.choice(np.float32([0.0, -0.0, 0.5, 1.0]), size=(B, L)).astype(np.float32)
+        s = np.where(np.arange(L)[None, :] < 3, np.float32(1.0), s)
+    elif case == "all_equal":
+        s = np.full((B, L), 0.75, np.float32)
+    elif case == "coarse_ties":
+        s = -np.sort(-(np.round(rng.beta(6.0, 2.0, size=(B, L)) * 4) / 4), axis=1).astype(np.float32)
+    else:
+        s = rng.beta(6.0, 2.0, size=(B, L)).astype(np.float32)
+    for budget in (B, B + 1, B * (L + 1) // 2, B * (L + 1) - 1, B * (L + 1) + 7):
+        ref = oracle.dvl_allocate(s, budget)
+        vl, off, sm = specv.dvl_allocate_pack(torch.from_numpy(s).cuda(), budget)
+        np.testing.assert_array_equal(_cpu(vl), ref["verify_len"])
+        np.testing.assert_array_equal(_cpu(off), ref["offsets"])
+        np.testing.assert_array_equal(_cpu(sm), ref["slot_map"])
 
 
 def test_dvl_flags_bad_scores():
