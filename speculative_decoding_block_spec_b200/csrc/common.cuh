@@ -4,19 +4,6 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "exp2_fma.cuh"
-
-// Exponentials per 16-byte vector of logits that the streaming fold computes
-// on the FMA pipe (exp2_fma) instead of the MUFU unit: the last ones of its
-// 8 bf16 or 4 fp32 elements. The share balances the two pipes so that
-// neither caps the HBM stream.
-#ifndef SPECV_FMA_EXP_BF16
-#define SPECV_FMA_EXP_BF16 2
-#endif
-#ifndef SPECV_FMA_EXP_F32
-#define SPECV_FMA_EXP_F32 1
-#endif
-
 namespace specv {
 
 constexpr int kThreads = 256;          // threads per block, every kernel
@@ -205,7 +192,7 @@ __device__ __forceinline__ int block_exclusive_scan(int* arr, int n, int* tmp) {
 
 // Fold N 16-byte vectors into the running (m, s): the group maximum exactly
 // (raw bf16 pairs), a rescale of s when it grows, then one base-2
-// exponential per element, kFma of each vector's on the FMA pipe.
+// exponential per element.
 template <int DT, int N>
 __device__ __forceinline__ void fold_vectors(const uint4 (&v)[N], float& m, float& s, float k) {
   constexpr int E = Elem<DT>::kPerVec;
@@ -234,11 +221,9 @@ __device__ __forceinline__ void fold_vectors(const uint4 (&v)[N], float& m, floa
   for (int t = 0; t < N; ++t) {
     float x[E];
     Elem<DT>::unpack(v[t], x);
-    constexpr int kFma = DT == 1 ? SPECV_FMA_EXP_BF16 : SPECV_FMA_EXP_F32;
-    static_assert(kFma >= 0 && kFma <= E, "FMA-pipe share out of range");
     float e[E];
 #pragma unroll
-    for (int i = 0; i < E; ++i) e[i] = i >= E - kFma ? exp2_fma((x[i] - m) * k) : ex2((x[i] - m) * k);
+    for (int i = 0; i < E; ++i) e[i] = ex2((x[i] - m) * k);
 #pragma unroll
     for (int w = 1; w < E; w <<= 1)
 #pragma unroll

@@ -15,13 +15,15 @@
 //  1. one thread per request forms its products in fp64, left to right, and
 //     stores them as 64-bit keys whose unsigned order is the order of P
 //     (+0 and -0 are one key, as they compare equal);
-//  2. a radix select over the keys, eight 8-bit digits from the top, finds
-//     the key K of the (budget' - B)-th entry in the order (P desc, flat
-//     index asc): per digit a 256-bin histogram of the entries that still
-//     match the prefix, and one warp's suffix scan over it;
-//  3. entries with key > K are selected, and of those equal to K the first
-//     ones by flat index (an exclusive scan over the equal-key flags, only
-//     when some entries share K and not all of them are taken);
+//  2. a radix select over the keys, 8-bit digits from the top, finds the
+//     (budget' - B)-th entry in the order (P desc, flat index asc): per digit
+//     a 256-bin histogram of the entries that still match the prefix (one
+//     shared atomic per distinct digit of a warp, grouped with
+//     __match_any_sync) and one warp's suffix scan over it; the descent
+//     stops at the first digit whose bin is taken whole;
+//  3. entries above the cut are selected, and of those equal to it the
+//     first ones by flat index (an exclusive scan over the equal-key flags,
+//     only when equal full keys straddle the cut);
 //  4. verify_len[b] = selected entries of row b; an exclusive scan of
 //     verify_len + 1 gives the offsets, from which the slot map is filled.
 // O(B L) work per digit; k_dvl_pack then copies the selected dense target
@@ -35,6 +37,7 @@ namespace specv {
 
 constexpr int kDvlThreads = 1024;
 constexpr int kDvlWarps = kDvlThreads / 32;
+constexpr int kDvlMaxL = 32;  // SPEC_MAX_L
 
 // Order-preserving key of a product: unsigned order of the key = numeric
 // order of P (negative values below +0; -0 maps to the key of +0; a NaN,
@@ -51,7 +54,7 @@ __global__ void __launch_bounds__(kDvlThreads, 1) k_dvl_allocate(const float* __
   extern __shared__ unsigned long long sKey[];  // [B*L] keys, then int[B*L] equal-key ranks, int[B + 1] lengths
   __shared__ int s_hist[256];
   __shared__ int s_tmp[kDvlWarps + 1];
-  __shared__ int s_digit, s_k, s_eq, s_flag;
+  __shared__ int s_digit, s_k, s_binc, s_flag;
   pdl_wait();
   pdl_trigger();
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -59,36 +62,46 @@ __global__ void __launch_bounds__(kDvlThreads, 1) k_dvl_allocate(const float* __
   int* sRank = reinterpret_cast<int*>(sKey + n);  // index-order rank among the entries equal to the cut key
   int* lens = sRank + n;                           // verify_len + 1, then offsets
 
-  if (tid == 0) {
-    s_flag = 0;
-    s_eq = 0;
-  }
+  if (tid == 0) s_flag = 0;
   __syncthreads();
   int bad = 0;
   for (int r = tid; r < B; r += kDvlThreads) {
+    float sv[kDvlMaxL];
+#pragma unroll
+    for (int i = 0; i < kDvlMaxL; ++i) sv[i] = i < L ? scores[static_cast<int64_t>(r) * L + i] : 1.f;
     double P = 1.0;
-    for (int i = 0; i < L; ++i) {
-      const float s = scores[static_cast<int64_t>(r) * L + i];
-      bad |= !(s >= 0.f && s <= 1.f);
-      P = P * static_cast<double>(s);
-      sKey[r * L + i] = p_key(P);
+#pragma unroll
+    for (int i = 0; i < kDvlMaxL; ++i) {
+      if (i < L) {
+        bad |= !(sv[i] >= 0.f && sv[i] <= 1.f);
+        P = P * static_cast<double>(sv[i]);
+        sKey[r * L + i] = p_key(P);
+      }
     }
   }
   if (bad) atomicOr(&s_flag, kFlagScores);
+  __syncthreads();
 
   const int64_t cap = static_cast<int64_t>(B) * (L + 1);
   const int take = static_cast<int>(std::min<int64_t>(budget, cap)) - B;  // 0 <= take <= n
-  unsigned long long kth = ~0ull;  // take == 0: nothing is selected (no key exceeds ~0)
-  int k_eq = 0;                    // entries equal to kth that are taken
+  // The cut: entries whose key, under `mask`, is above `prefix` are selected; of those equal to it under the
+  // mask, all are selected when the bin holds exactly the k still wanted, else (equal full keys) the first k
+  // by flat index. take == 0 selects nothing: no masked key exceeds the all-ones prefix.
+  unsigned long long prefix = ~0ull, mask = ~0ull;
+  int k = 0, binc = 0;
   if (take > 0) {
-    unsigned long long prefix = 0, mask = 0;
-    int k = take;  // rank (1-based, descending) of the wanted entry among those matching the prefix
+    prefix = 0ull;
+    mask = 0ull;
+    k = take;  // rank (1-based, descending) of the wanted entry among those matching the prefix
     for (int shift = 56; shift >= 0; shift -= 8) {
       if (tid < 256) s_hist[tid] = 0;
       __syncthreads();
-      for (int e = tid; e < n; e += kDvlThreads) {
-        const unsigned long long u = sKey[e];
-        if ((u & mask) == prefix) atomicAdd(&s_hist[(u >> shift) & 255], 1);
+      for (int base = wid * 32; base < n; base += kDvlThreads) {  // warp-uniform trips: full-warp intrinsics
+        const int e = base + lane;
+        const unsigned long long u = e < n ? sKey[e] : 0ull;
+        const int d = (e < n && (u & mask) == prefix) ? static_cast<int>((u >> shift) & 255) : 256;
+        const unsigned peers = __match_any_sync(0xffffffffu, d);  // one atomic per distinct digit of the warp
+        if (d < 256 && lane == __ffs(peers) - 1) atomicAdd(&s_hist[d], __popc(peers));
       }
       __syncthreads();
       if (wid == 0) {  // lane l owns digits 255 - 8l ... 248 - 8l (descending)
@@ -98,7 +111,7 @@ __global__ void __launch_bounds__(kDvlThreads, 1) k_dvl_allocate(const float* __
           c[t] = s_hist[255 - 8 * lane - t];
           sum += c[t];
         }
-        int incl = sum;  // inclusive scan over lanes: entries in digits above and including this lane's
+        int incl = sum;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const int v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -112,29 +125,26 @@ __global__ void __launch_bounds__(kDvlThreads, 1) k_dvl_allocate(const float* __
             if (run < k && run + c[t] >= k) {
               s_digit = 255 - 8 * lane - t;
               s_k = k - run;
+              s_binc = c[t];
             }
             run += c[t];
           }
         }
       }
       __syncthreads();
-      // s_digit and s_k are rewritten only after two more barriers of the next digit
+      // s_digit, s_k and s_binc are rewritten only after two more barriers of the next digit
       prefix |= static_cast<unsigned long long>(s_digit) << shift;
       mask |= 255ull << shift;
       k = s_k;
+      binc = s_binc;
+      if (binc == k) break;  // the whole bin is taken: nothing below this digit matters (block-uniform)
     }
-    kth = prefix;
-    k_eq = k;
   }
 
-  // entries equal to kth: the first k_eq of them by flat index are taken
-  int n_eq_local = 0;
-  for (int e = tid; e < n; e += kDvlThreads) n_eq_local += sKey[e] == kth;
-  if (n_eq_local) atomicAdd(&s_eq, n_eq_local);
-  __syncthreads();
-  const bool rank_eq = s_eq > k_eq && k_eq > 0;  // only then does the index order among equals matter
+  // entries equal to the cut under the mask: all taken, or (ties of full keys) the first k by flat index
+  const bool rank_eq = take > 0 && binc > k;
   if (rank_eq) {
-    for (int e = tid; e < n; e += kDvlThreads) sRank[e] = sKey[e] == kth;
+    for (int e = tid; e < n; e += kDvlThreads) sRank[e] = (sKey[e] & mask) == prefix;
     __syncthreads();
     block_exclusive_scan<kDvlThreads>(sRank, n, s_tmp);
   }
@@ -143,8 +153,8 @@ __global__ void __launch_bounds__(kDvlThreads, 1) k_dvl_allocate(const float* __
     int ell = 0;
     for (int i = 0; i < L; ++i) {
       const int e = r * L + i;
-      const unsigned long long u = sKey[e];
-      ell += (u > kth || (u == kth && (rank_eq ? sRank[e] < k_eq : k_eq > 0))) ? 1 : 0;
+      const unsigned long long um = sKey[e] & mask;
+      ell += (um > prefix || (um == prefix && take > 0 && (rank_eq ? sRank[e] < k : true))) ? 1 : 0;
     }
     verify_len[r] = ell;
     lens[r] = ell + 1;

@@ -13,23 +13,30 @@
 // and the nucleus is fixed by a cut: the logit value x_c and token v_c of its
 // last member; token v is kept iff x_v > x_c, or x_v == x_c and v <= v_c.
 //
-// k_nucleus, one row at a time per block (rows strided over the grid):
+// k_nucleus, one row at a time per block (one block per SM, rows strided over
+// the grid):
 //  1. the row's maximum m from the statistics partials;
-//  2. a radix descent over 32-bit order keys of the logits (bf16 logits
-//     widened exactly to fp32): per digit, a shared-memory histogram of the
-//     mass of the tokens that match the key prefix found so far, then a
-//     descending scan for the digit whose bin carries the running mass
-//     across top_p * total. Digits: bits 31..20 (4096 bins), then 19..16 for
-//     bf16 (whose low 16 bits are fixed by the sign), or 19..8 and 7..0 for
-//     fp32. Masses are 2^((x - m) k) in fixed point (scaled by 2^42, rounded
-//     to the nearest unit) summed with 64-bit integer atomics, so every sum
-//     is exact and independent of the order the atomics land in;
+//  2. bf16 rows: one pass counts the tokens of every bf16 value (65,536
+//     16-bit counters packed two to a 32-bit word in shared memory, native
+//     integer atomics, no exponential per token); then the warps walk the
+//     values from the largest down, each value's mass being its count times
+//     2^((x - m) k) in fixed point (scaled by 2^42, rounded), and find the
+//     value whose mass carries the running total across top_p * total.
+//     Sums are exact integers, so the cut does not depend on the order of
+//     any addition. A row whose counters could have overflowed (their total
+//     is not V) takes the radix path instead;
+//     fp32 rows: a radix descent over 32-bit order keys of the logits, per
+//     digit a shared-memory histogram of the fixed-point mass of the tokens
+//     that match the key prefix found so far (64-bit integer atomics) and a
+//     descending scan for the crossing digit: bits 31..20, 19..8, 7..0 (the
+//     last digit also counts tokens);
 //  3. at the cut value, the number n of its tokens needed to reach top_p;
 //     if not all of them are needed, the n-th such token in index order is
 //     found with a warp-ordered count (the tie cut);
 //  4. outputs: m, the log of the nucleus mass sum_{v kept} 2^((x_v - m) k)
 //     (the filtered rows' normaliser), the cut key and the cut token.
-// The first digit streams the row from HBM; the later passes find it in L2.
+// The counting pass streams the row from HBM; the tie cut re-reads it from
+// L2.
 #include <algorithm>
 
 #include "common.cuh"
@@ -38,10 +45,11 @@
 
 namespace specv {
 
-constexpr int kNucThreads = 512;
+constexpr int kNucThreads = 1024;
 constexpr int kNucWarps = kNucThreads / 32;
 constexpr int kFix = 42;              // fixed-point scale of the masses: sums of up to 2^20 terms of <= 1 fit 2^62
-constexpr int kNucBins = 4096;        // bins of the widest digit
+constexpr int kNucBins = 4096;        // bins of the widest radix digit
+constexpr int kValueWords = 32768;    // bf16: 65,536 16-bit counters, two per word
 constexpr int kNucCountBins = 256;    // bins of the last digit, which also counts tokens
 
 // round(q * 2^kFix) for q in [0, 1] (fp32 bits; no conversion instruction).
@@ -91,7 +99,7 @@ __device__ __forceinline__ void digit_pass(const char* row, int64_t V, float m, 
                                            uint32_t pmask, int shift, uint32_t dmask, bool count,
                                            unsigned long long* hist, unsigned* cnt) {
   constexpr int E = VEC ? Elem<DT>::kPerVec : 1;
-  constexpr int U = VEC ? 2 : 1;  // units in flight per thread
+  constexpr int U = VEC ? 2 : 1;  // units in flight per thread (the radix path is the rare one)
   const int64_t Vu = V / E;
   for (int64_t u0 = threadIdx.x; u0 < Vu; u0 += U * kNucThreads) {
     float x[U][E];
@@ -207,19 +215,157 @@ __device__ __forceinline__ int64_t nth_equal(const char* row, int64_t V, uint32_
   return *s_v;
 }
 
+// Order key of a bf16 logit from its 16 bits (as order_key of the widened
+// value, shifted down 16), and the value of a key.
+__device__ __forceinline__ uint32_t order_key16(uint32_t h) {
+  h &= 0xFFFFu;
+  if (h == 0x8000u) h = 0u;
+  return (h & 0x8000u) ? (~h & 0xFFFFu) : (h | 0x8000u);
+}
+__device__ __forceinline__ float key16_value(uint32_t key) {
+  const uint32_t h = (key & 0x8000u) ? (key & 0x7FFFu) : (~key & 0xFFFFu);
+  return __uint_as_float(h << 16);
+}
+// The widened value's 32-bit order key: its low half is fixed by the sign.
+__device__ __forceinline__ uint32_t key16_to_key32(uint32_t key) {
+  return (key << 16) | ((key & 0x8000u) ? 0u : 0xFFFFu);
+}
+
+// bf16: count the tokens of every value (counter key in half key >> 1 of the
+// word array; low half for even keys).
+template <bool VEC>
+__device__ __forceinline__ void count_values(const char* row, int64_t V, uint32_t* cnt) {
+  if constexpr (VEC) {
+    constexpr int U = 4;
+    const int64_t Vu = V / 8;
+    for (int64_t u0 = threadIdx.x; u0 < Vu; u0 += U * kNucThreads) {
+      uint4 w[U];
+#pragma unroll
+      for (int h = 0; h < U; ++h) {
+        const int64_t u = u0 + static_cast<int64_t>(h) * kNucThreads;
+        w[h] = u < Vu ? ldg16(reinterpret_cast<const uint4*>(row) + u) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int h = 0; h < U; ++h) {
+        if (u0 + static_cast<int64_t>(h) * kNucThreads >= Vu) break;
+        const uint32_t ws[4] = {w[h].x, w[h].y, w[h].z, w[h].w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const uint32_t key = order_key16(ws[c] >> (16 * half));
+            atomicAdd(&cnt[key >> 1], (key & 1u) ? 0x10000u : 1u);
+          }
+        }
+      }
+    }
+  } else {
+    const unsigned short* r16 = reinterpret_cast<const unsigned short*>(row);
+    for (int64_t v = threadIdx.x; v < V; v += kNucThreads) {
+      const uint32_t key = order_key16(__ldg(r16 + v));
+      atomicAdd(&cnt[key >> 1], (key & 1u) ? 0x10000u : 1u);
+    }
+  }
+}
+
+// Tokens and fixed-point mass of the two keys of counter word `word`
+// (higher key first).
+__device__ __forceinline__ void word_mass(const uint32_t* cnt, int word, float m, float k, uint32_t (&c)[2],
+                                          unsigned long long (&mass)[2]) {
+  const uint32_t wv = cnt[word];
+  c[0] = wv >> 16;       // key 2 word + 1
+  c[1] = wv & 0xFFFFu;   // key 2 word
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    mass[t] = 0ull;
+    if (c[t]) {
+      const uint32_t key = 2u * static_cast<uint32_t>(word) + 1u - t;
+      mass[t] = static_cast<unsigned long long>(c[t]) * to_fixed(ex2((key16_value(key) - m) * k));
+    }
+  }
+}
+
+// Radix descent (fp32 rows, and bf16 rows whose counters could have
+// overflowed): the cut key kappa, the mass above it, the row's whole mass and
+// the target; also the tokens at the cut value (c) and the mass of each
+// (each). Called by the whole block; `hist` is 4096 64-bit bins.
 template <int DT, bool VEC>
-__global__ void __launch_bounds__(kNucThreads, 2) k_nucleus(NucleusArgs a) {
-  extern __shared__ unsigned long long nuc_smem[];  // hist[kNucBins], then walk rowoff[B + 1], base[B]
+__device__ __forceinline__ void radix_cut(const char* row, int64_t V, float m, float k, double top_p,
+                                          unsigned long long* hist, unsigned* s_cnt, unsigned long long* s_tmp,
+                                          int* s_d, unsigned long long* s_above, unsigned long long& whole,
+                                          unsigned long long& target, unsigned long long& above, uint32_t& kappa,
+                                          unsigned& c, unsigned long long& each) {
+  const int tid = threadIdx.x;
+  constexpr bool bf16 = DT == 1;
+  for (int i = tid; i < kNucBins; i += kNucThreads) hist[i] = 0ull;
+  for (int i = tid; i < kNucCountBins; i += kNucThreads) s_cnt[i] = 0u;
+  __syncthreads();
+  // digit 1: bits 31..20, every token; its total is the row's whole mass
+  digit_pass<DT, VEC>(row, V, m, k, 0u, 0u, 20, 0xFFFu, false, hist, s_cnt);
+  __syncthreads();
+  unsigned long long local = 0;
+  for (int i = tid; i < kNucBins; i += kNucThreads) local += hist[i];
+  const unsigned long long excl = block_scan_u64(local, s_tmp);
+  if (tid == kNucThreads - 1) *s_above = excl + local;
+  __syncthreads();
+  whole = *s_above;
+  target = static_cast<unsigned long long>(ceil(top_p * static_cast<double>(whole)));
+  if (target < 1ull) target = 1ull;
+  if (target > whole) target = whole;
+  __syncthreads();
+  find_digit(hist, kNucBins, 0ull, target, s_tmp, s_d, s_above);
+  uint32_t prefix = static_cast<uint32_t>(*s_d) << 20, pmask = 0xFFF00000u;
+  above = *s_above;
+  const int shift = bf16 ? 16 : 8;      // digit 2: bits 19..16 complete a widened bf16 key; fp32: 19..8
+  const int nb = bf16 ? 16 : kNucBins;
+  __syncthreads();
+  for (int i = tid; i < kNucBins; i += kNucThreads) hist[i] = 0ull;
+  __syncthreads();
+  digit_pass<DT, VEC>(row, V, m, k, prefix, pmask, shift, static_cast<uint32_t>(nb - 1), bf16, hist, s_cnt);
+  __syncthreads();
+  find_digit(hist, nb, above, target, s_tmp, s_d, s_above);
+  int dl = *s_d;
+  prefix |= static_cast<uint32_t>(dl) << shift;
+  above = *s_above;
+  if (bf16) {
+    kappa = prefix | ((prefix & 0x80000000u) ? 0u : 0xFFFFu);  // the low half of a widened bf16 key
+  } else {  // digit 3: bits 7..0, with token counts
+    __syncthreads();
+    for (int i = tid; i < kNucCountBins; i += kNucThreads) hist[i] = 0ull;
+    __syncthreads();
+    digit_pass<DT, VEC>(row, V, m, k, prefix, 0xFFFFFF00u, 0, 0xFFu, true, hist, s_cnt);
+    __syncthreads();
+    find_digit(hist, kNucCountBins, above, target, s_tmp, s_d, s_above);
+    dl = *s_d;
+    above = *s_above;
+    kappa = prefix | static_cast<uint32_t>(dl);
+  }
+  // (the crossing bin holds mass, hence at least one token; the guards only keep every division defined)
+  c = s_cnt[dl];
+  each = c ? hist[dl] / c : 1ull;  // every token of the cut value has the same mass
+  __syncthreads();
+}
+
+template <int DT, bool VEC>
+__global__ void __launch_bounds__(kNucThreads, 1) k_nucleus(NucleusArgs a) {
+  // dynamic shared memory: a 128 KiB region (bf16 value counters, or the
+  // radix path's 4096 64-bit bins), then the walk (rowoff[B + 1], base[B])
+  extern __shared__ unsigned long long nuc_smem[];
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(nuc_smem);
   unsigned long long* hist = nuc_smem;
-  int* walk_smem = reinterpret_cast<int*>(nuc_smem + kNucBins);
+  int* walk_smem = reinterpret_cast<int*>(nuc_smem + kValueWords / 2);
   __shared__ unsigned s_cnt[kNucCountBins];
   __shared__ unsigned long long s_tmp[kNucWarps + 1];
   __shared__ int s_itmp[kNucWarps + 1];
   __shared__ unsigned s_wc[kNucWarps];
+  __shared__ unsigned long long s_wmass[kNucWarps];
+  __shared__ unsigned s_wtok[kNucWarps];
   __shared__ float s_m;
   __shared__ const char* s_row;
   __shared__ int s_d;
-  __shared__ unsigned long long s_above;
+  __shared__ unsigned long long s_above, s_each;
+  __shared__ unsigned s_c;
+  __shared__ uint32_t s_kappa;
   __shared__ long long s_v;
   pdl_wait();
   pdl_trigger();
@@ -227,8 +373,7 @@ __global__ void __launch_bounds__(kNucThreads, 2) k_nucleus(NucleusArgs a) {
   const Walk w{walk_smem, walk_smem + rs.B + 1};
   const int64_t nrows = build_walk<kNucThreads>(rs, walk_smem, s_itmp);
   const int64_t N = nrows * a.Vu;
-  const int tid = threadIdx.x;
-  const bool bf16 = DT == 1;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   for (int64_t r = blockIdx.x; r < nrows; r += gridDim.x) {
     if (tid == 0) {
       float m, s;
@@ -237,8 +382,6 @@ __global__ void __launch_bounds__(kNucThreads, 2) k_nucleus(NucleusArgs a) {
       const int32_t* tokp;
       s_row = locate<DT>(rs, w, r, tokp);
     }
-    for (int i = tid; i < kNucBins; i += kNucThreads) hist[i] = 0ull;
-    for (int i = tid; i < kNucCountBins; i += kNucThreads) s_cnt[i] = 0u;
     __syncthreads();
     const float m = s_m;
     const char* row = s_row;
@@ -252,63 +395,99 @@ __global__ void __launch_bounds__(kNucThreads, 2) k_nucleus(NucleusArgs a) {
       __syncthreads();
       continue;
     }
-    // digit 1: bits 31..20, every token; its total is the row's whole mass
-    digit_pass<DT, VEC>(row, a.V, m, a.k, 0u, 0u, 20, 0xFFFu, false, hist, s_cnt);
-    __syncthreads();
-    unsigned long long local = 0;
-    for (int i = tid; i < kNucBins; i += kNucThreads) local += hist[i];
-    const unsigned long long total = block_scan_u64(local, s_tmp) + local;  // the last thread's inclusive sum
-    if (tid == kNucThreads - 1) s_above = total;
-    __syncthreads();
-    const unsigned long long whole = s_above;
-    unsigned long long target = static_cast<unsigned long long>(ceil(a.top_p * static_cast<double>(whole)));
-    if (target < 1ull) target = 1ull;
-    if (target > whole) target = whole;
-    __syncthreads();
-    find_digit(hist, kNucBins, 0ull, target, s_tmp, &s_d, &s_above);
-    uint32_t prefix = static_cast<uint32_t>(s_d) << 20, pmask = 0xFFF00000u;
-    unsigned long long above = s_above;
-    int nb, shift;
-    if (bf16) {  // digit 2: bits 19..16, which complete a widened bf16 key
-      shift = 16;
-      nb = 16;
-    } else {     // digit 2: bits 19..8
-      shift = 8;
-      nb = kNucBins;
+    unsigned long long whole = 0, target = 0, above = 0, each = 1;
+    unsigned c = 0;
+    uint32_t kappa = 0;
+    bool radix = DT == 0;
+    if constexpr (DT == 1) {
+      for (int i = tid; i < kValueWords; i += kNucThreads) cnt[i] = 0u;
+      __syncthreads();
+      count_values<VEC>(row, a.V, cnt);
+      __syncthreads();
+      // warp wid walks counter words 32767 - 1024 wid down to 32767 - 1024 wid - 1023 (keys descending),
+      // 32 consecutive words per step, one per lane
+      const int wtop = kValueWords - 1 - 1024 * wid;
+      unsigned long long wm = 0;
+      unsigned wt = 0;
+      for (int st = 0; st < 32; ++st) {
+        uint32_t cc[2];
+        unsigned long long mm[2];
+        word_mass(cnt, wtop - 32 * st - lane, m, a.k, cc, mm);
+        wm += mm[0] + mm[1];
+        wt += cc[0] + cc[1];
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        wm += __shfl_xor_sync(0xffffffffu, wm, o);
+        wt += __shfl_xor_sync(0xffffffffu, wt, o);
+      }
+      if (lane == 0) {
+        s_wmass[wid] = wm;
+        s_wtok[wid] = wt;
+      }
+      if (tid == 0) s_c = 0u;
+      __syncthreads();
+      unsigned long long base = 0, all = 0;
+      unsigned tokens = 0;
+      for (int q = 0; q < kNucWarps; ++q) {
+        if (q < wid) base += s_wmass[q];
+        all += s_wmass[q];
+        tokens += s_wtok[q];
+      }
+      if (tokens != static_cast<unsigned>(a.V)) {
+        radix = true;  // a value with more than 65,535 tokens wrapped its counter
+      } else {
+        whole = all;
+        target = static_cast<unsigned long long>(ceil(a.top_p * static_cast<double>(whole)));
+        if (target < 1ull) target = 1ull;
+        if (target > whole) target = whole;
+        if (base < target && base + s_wmass[wid] >= target) {  // this warp's values hold the crossing
+          unsigned long long run = base;
+          for (int st = 0; st < 32; ++st) {
+            const int word = wtop - 32 * st - lane;
+            uint32_t cc[2];
+            unsigned long long mm[2];
+            word_mass(cnt, word, m, a.k, cc, mm);
+            const unsigned long long lm = mm[0] + mm[1];
+            unsigned long long incl = lm;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+              const unsigned long long t = __shfl_up_sync(0xffffffffu, incl, o);
+              if (lane >= o) incl += t;
+            }
+            const unsigned long long ex = run + incl - lm;  // mass of every larger value
+            if (ex < target && ex + mm[0] >= target) {  // the higher key of the word
+              s_kappa = 2u * static_cast<uint32_t>(word) + 1u;
+              s_above = ex;
+              s_c = cc[0];
+              s_each = mm[0] / cc[0];
+            } else if (ex + mm[0] < target && ex + lm >= target) {
+              s_kappa = 2u * static_cast<uint32_t>(word);
+              s_above = ex + mm[0];
+              s_c = cc[1];
+              s_each = mm[1] / cc[1];
+            }
+            run += __shfl_sync(0xffffffffu, incl, 31);
+            if (run >= target) break;
+          }
+        }
+        __syncthreads();
+        kappa = key16_to_key32(s_kappa);
+        above = s_above;
+        c = s_c;
+        each = s_each ? s_each : 1ull;
+      }
+      __syncthreads();
     }
-    __syncthreads();
-    for (int i = tid; i < kNucBins; i += kNucThreads) hist[i] = 0ull;
-    __syncthreads();
-    digit_pass<DT, VEC>(row, a.V, m, a.k, prefix, pmask, shift, static_cast<uint32_t>(nb - 1), bf16, hist, s_cnt);
-    __syncthreads();
-    find_digit(hist, nb, above, target, s_tmp, &s_d, &s_above);
-    int dl = s_d;
-    prefix |= static_cast<uint32_t>(dl) << shift;
-    above = s_above;
-    uint32_t kappa;
-    if (bf16) {
-      kappa = prefix | ((prefix & 0x80000000u) ? 0u : 0xFFFFu);  // the low half of a widened bf16 key
-    } else {     // digit 3: bits 7..0, with token counts
-      pmask = 0xFFFFFF00u;
-      __syncthreads();
-      for (int i = tid; i < kNucCountBins; i += kNucThreads) hist[i] = 0ull;
-      __syncthreads();
-      digit_pass<DT, VEC>(row, a.V, m, a.k, prefix, pmask, 0, 0xFFu, true, hist, s_cnt);
-      __syncthreads();
-      find_digit(hist, kNucCountBins, above, target, s_tmp, &s_d, &s_above);
-      dl = s_d;
-      above = s_above;
-      kappa = prefix | static_cast<uint32_t>(dl);
-    }
+    if (radix)
+      radix_cut<DT, VEC>(row, a.V, m, a.k, a.top_p, hist, s_cnt, s_tmp, &s_d, &s_above, whole, target, above,
+                         kappa, c, each);
     // tokens at the cut value: how many are needed, and which is the last
-    const unsigned c = s_cnt[dl];
-    const unsigned long long each = hist[dl] / c;  // every token of the cut value has the same mass
     const unsigned long long need = (target - above + each - 1) / each;
     const unsigned take = static_cast<unsigned>(need < c ? need : c);
     const unsigned long long kept = above + static_cast<unsigned long long>(take) * each;
-    __syncthreads();
     int64_t vcut = a.V - 1;
-    if (take < c) vcut = nth_equal<DT, VEC>(row, a.V, kappa, take, s_wc, &s_v);
+    if (take > 0 && take < c) vcut = nth_equal<DT, VEC>(row, a.V, kappa, take, s_wc, &s_v);
     if (tid == 0) {
       a.row_m[r] = m;
       a.row_lf[r] = log(static_cast<double>(kept)) - kFix * 0.6931471805599453;
@@ -320,17 +499,15 @@ __global__ void __launch_bounds__(kNucThreads, 2) k_nucleus(NucleusArgs a) {
 }
 
 cudaError_t launch_nucleus(const NucleusArgs& a, int dtype, bool vec, cudaStream_t st) {
-  const size_t smem = kNucBins * sizeof(unsigned long long) + static_cast<size_t>(2 * a.rs.B + 1) * sizeof(int);
+  const size_t smem = kValueWords * sizeof(uint32_t) + static_cast<size_t>(2 * a.rs.B + 1) * sizeof(int);
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t rows_max = static_cast<int64_t>(a.rs.B) * ((a.rs.K + 1) * a.rs.L + 1);
-  const dim3 grid(static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(rows_max, 3 * sms))));
+  const dim3 grid(static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(rows_max, sms))));
   auto go = [&](auto kernel) {
-    if (smem > 48 * 1024) {
-      const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-    }
+    const cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
     return launch_pdl(kernel, grid, dim3(kNucThreads), smem, st, a);
   };
   if (dtype == 0) return vec ? go(k_nucleus<0, true>) : go(k_nucleus<0, false>);
