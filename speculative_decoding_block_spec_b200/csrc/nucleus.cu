@@ -165,14 +165,33 @@ __device__ __forceinline__ int64_t nth_equal(const char* row, int64_t V, uint32_
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int64_t cw = (Vu + kNucWarps - 1) / kNucWarps;  // units per warp, contiguous
   const int64_t a = min(Vu, w * cw), b = min(Vu, a + cw);
+  // bf16 vectors compare raw bit pairs: the raw bits of the cut value (and
+  // those of -0 when the cut value is zero) in both halves of a word
+  const uint32_t k16 = kappa >> 16;
+  const uint32_t hraw = (k16 & 0x8000u) ? (k16 & 0x7FFFu) : (~k16 & 0xFFFFu);
+  const uint32_t hh = hraw | (hraw << 16);
+  const bool zero = hraw == 0u;
   auto matches = [&](int64_t u) -> unsigned {  // bit e set when element e of unit u has key kappa
-    float x[E];
-    if constexpr (VEC) Elem<DT>::unpack(ldg16(reinterpret_cast<const uint4*>(row) + u), x);
-    else x[0] = Elem<DT>::at(row, u);
-    unsigned bits = 0;
+    if constexpr (DT == 1 && VEC) {
+      const uint4 q = ldg16(reinterpret_cast<const uint4*>(row) + u);
+      const uint32_t ws[4] = {q.x, q.y, q.z, q.w};
+      unsigned bits = 0;
 #pragma unroll
-    for (int e = 0; e < E; ++e) bits |= (order_key(x[e]) == kappa ? 1u : 0u) << e;
-    return bits;
+      for (int c = 0; c < 4; ++c) {
+        uint32_t eq = __vcmpeq2(ws[c], hh);
+        if (zero) eq |= __vcmpeq2(ws[c], 0x80008000u);
+        bits |= ((eq & 1u) << (2 * c)) | (((eq >> 16) & 1u) << (2 * c + 1));
+      }
+      return bits;
+    } else {
+      float x[E];
+      if constexpr (VEC) Elem<DT>::unpack(ldg16(reinterpret_cast<const uint4*>(row) + u), x);
+      else x[0] = Elem<DT>::at(row, u);
+      unsigned bits = 0;
+#pragma unroll
+      for (int e = 0; e < E; ++e) bits |= (order_key(x[e]) == kappa ? 1u : 0u) << e;
+      return bits;
+    }
   };
   if (threadIdx.x == 0) *s_v = V - 1;  // overwritten by the lane that finds the token
   unsigned c = 0;
@@ -231,8 +250,16 @@ __device__ __forceinline__ uint32_t key16_to_key32(uint32_t key) {
   return (key << 16) | ((key & 0x8000u) ? 0u : 0xFFFFu);
 }
 
-// bf16: count the tokens of every value (counter key in half key >> 1 of the
-// word array; low half for even keys).
+// Order keys of the two bf16 values packed in a 32-bit word (each half as
+// order_key16 of its half): negative h -> ~h, non-negative h -> h | 0x8000,
+// and -0 takes the key of +0.
+__device__ __forceinline__ uint32_t order_keys2(uint32_t w) {
+  const uint32_t neg = ((w >> 15) & 0x00010001u) * 0x7FFFu;  // 0x7FFF in each negative half
+  return (w ^ (neg | 0x80008000u)) ^ __vcmpeq2(w, 0x80008000u);
+}
+
+// bf16: count the tokens of every value (the counter of key v is half v & 1
+// of word v >> 1: the low half for even keys).
 template <bool VEC>
 __device__ __forceinline__ void count_values(const char* row, int64_t V, uint32_t* cnt) {
   if constexpr (VEC) {
@@ -251,11 +278,9 @@ __device__ __forceinline__ void count_values(const char* row, int64_t V, uint32_
         const uint32_t ws[4] = {w[h].x, w[h].y, w[h].z, w[h].w};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const uint32_t key = order_key16(ws[c] >> (16 * half));
-            atomicAdd(&cnt[key >> 1], (key & 1u) ? 0x10000u : 1u);
-          }
+          const uint32_t key = order_keys2(ws[c]);
+          atomicAdd(&cnt[(key >> 1) & 0x7FFFu], 1u << ((key & 1u) << 4));
+          atomicAdd(&cnt[key >> 17], 1u << (((key >> 16) & 1u) << 4));
         }
       }
     }
@@ -358,8 +383,9 @@ __global__ void __launch_bounds__(kNucThreads, 1) k_nucleus(NucleusArgs a) {
   __shared__ unsigned long long s_tmp[kNucWarps + 1];
   __shared__ int s_itmp[kNucWarps + 1];
   __shared__ unsigned s_wc[kNucWarps];
-  __shared__ unsigned long long s_wmass[kNucWarps];
+  __shared__ unsigned long long s_step[kNucThreads];  // bf16: mass of each 32-word step, descending keys
   __shared__ unsigned s_wtok[kNucWarps];
+  __shared__ int s_sel;
   __shared__ float s_m;
   __shared__ const char* s_row;
   __shared__ int s_d;
@@ -375,12 +401,24 @@ __global__ void __launch_bounds__(kNucThreads, 1) k_nucleus(NucleusArgs a) {
   const int64_t N = nrows * a.Vu;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   for (int64_t r = blockIdx.x; r < nrows; r += gridDim.x) {
-    if (tid == 0) {
-      float m, s;
-      merge_row(a.part, r, a.Vu, N, a.G, a.k, m, s);
-      s_m = (isfinite(m) && isfinite(s)) ? m : NAN;
-      const int32_t* tokp;
-      s_row = locate<DT>(rs, w, r, tokp);
+    if (wid == 0) {  // the row maximum: the lanes load its partials in parallel (any order: a maximum)
+      const int64_t c0 = split_owner(r * a.Vu, N, a.G), c1 = split_owner((r + 1) * a.Vu - 1, N, a.G);
+      float mx = -INFINITY;
+      bool bad = false;
+      for (int64_t c = c0 + lane; c <= c1; c += 32) {
+        if (split_start(c + 1, N, a.G) == split_start(c, N, a.G)) continue;  // empty share: no partial
+        const float2 pr = __ldcg(a.part + c + r);
+        bad |= (pr.x != pr.x) || !isfinite(pr.y);
+        mx = fmaxf(mx, pr.x);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      bad = __any_sync(0xffffffffu, bad);
+      if (lane == 0) {
+        s_m = (!bad && isfinite(mx)) ? mx : NAN;
+        const int32_t* tokp;
+        s_row = locate<DT>(rs, w, r, tokp);
+      }
     }
     __syncthreads();
     const float m = s_m;
@@ -400,75 +438,76 @@ __global__ void __launch_bounds__(kNucThreads, 1) k_nucleus(NucleusArgs a) {
     uint32_t kappa = 0;
     bool radix = DT == 0;
     if constexpr (DT == 1) {
-      for (int i = tid; i < kValueWords; i += kNucThreads) cnt[i] = 0u;
+      for (int i = tid; i < kValueWords / 4; i += kNucThreads) reinterpret_cast<uint4*>(cnt)[i] = make_uint4(0, 0, 0, 0);
       __syncthreads();
       count_values<VEC>(row, a.V, cnt);
       __syncthreads();
-      // warp wid walks counter words 32767 - 1024 wid down to 32767 - 1024 wid - 1023 (keys descending),
-      // 32 consecutive words per step, one per lane
-      const int wtop = kValueWords - 1 - 1024 * wid;
-      unsigned long long wm = 0;
+      // step t = 32 wid + st covers counter words 32767 - 32 t down to 32767 - 32 t - 31 (keys descending),
+      // one word per lane; first the mass of every step, then a block scan over the 1024 steps, then the
+      // one step that holds the crossing
       unsigned wt = 0;
       for (int st = 0; st < 32; ++st) {
+        const int t = 32 * wid + st;
         uint32_t cc[2];
         unsigned long long mm[2];
-        word_mass(cnt, wtop - 32 * st - lane, m, a.k, cc, mm);
-        wm += mm[0] + mm[1];
+        word_mass(cnt, kValueWords - 1 - 32 * t - lane, m, a.k, cc, mm);
+        unsigned long long sm = mm[0] + mm[1];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
+        if (lane == 0) s_step[t] = sm;
         wt += cc[0] + cc[1];
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        wm += __shfl_xor_sync(0xffffffffu, wm, o);
-        wt += __shfl_xor_sync(0xffffffffu, wt, o);
+      for (int o = 16; o > 0; o >>= 1) wt += __shfl_xor_sync(0xffffffffu, wt, o);
+      if (lane == 0) s_wtok[wid] = wt;
+      if (tid == 0) {
+        s_c = 0u;
+        s_sel = 0;
       }
-      if (lane == 0) {
-        s_wmass[wid] = wm;
-        s_wtok[wid] = wt;
-      }
-      if (tid == 0) s_c = 0u;
       __syncthreads();
-      unsigned long long base = 0, all = 0;
+      const unsigned long long mine = s_step[tid];
+      const unsigned long long ex = block_scan_u64(mine, s_tmp);
+      if (tid == kNucThreads - 1) s_above = ex + mine;  // the whole mass
       unsigned tokens = 0;
-      for (int q = 0; q < kNucWarps; ++q) {
-        if (q < wid) base += s_wmass[q];
-        all += s_wmass[q];
-        tokens += s_wtok[q];
-      }
+      for (int q = 0; q < kNucWarps; ++q) tokens += s_wtok[q];
+      __syncthreads();
+      whole = s_above;
       if (tokens != static_cast<unsigned>(a.V)) {
         radix = true;  // a value with more than 65,535 tokens wrapped its counter
       } else {
-        whole = all;
         target = static_cast<unsigned long long>(ceil(a.top_p * static_cast<double>(whole)));
         if (target < 1ull) target = 1ull;
         if (target > whole) target = whole;
-        if (base < target && base + s_wmass[wid] >= target) {  // this warp's values hold the crossing
-          unsigned long long run = base;
-          for (int st = 0; st < 32; ++st) {
-            const int word = wtop - 32 * st - lane;
-            uint32_t cc[2];
-            unsigned long long mm[2];
-            word_mass(cnt, word, m, a.k, cc, mm);
-            const unsigned long long lm = mm[0] + mm[1];
-            unsigned long long incl = lm;
+        __syncthreads();  // every thread has read the whole mass from s_above
+        if (ex < target && ex + mine >= target) {  // this step holds the crossing
+          s_sel = tid;
+          s_above = ex;
+        }
+        __syncthreads();
+        if (wid == 0) {  // walk the one step: a warp scan over its 32 words
+          const int word = kValueWords - 1 - 32 * s_sel - lane;
+          uint32_t cc[2];
+          unsigned long long mm[2];
+          word_mass(cnt, word, m, a.k, cc, mm);
+          const unsigned long long lm = mm[0] + mm[1];
+          unsigned long long incl = lm;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-              const unsigned long long t = __shfl_up_sync(0xffffffffu, incl, o);
-              if (lane >= o) incl += t;
-            }
-            const unsigned long long ex = run + incl - lm;  // mass of every larger value
-            if (ex < target && ex + mm[0] >= target) {  // the higher key of the word
-              s_kappa = 2u * static_cast<uint32_t>(word) + 1u;
-              s_above = ex;
-              s_c = cc[0];
-              s_each = mm[0] / cc[0];
-            } else if (ex + mm[0] < target && ex + lm >= target) {
-              s_kappa = 2u * static_cast<uint32_t>(word);
-              s_above = ex + mm[0];
-              s_c = cc[1];
-              s_each = mm[1] / cc[1];
-            }
-            run += __shfl_sync(0xffffffffu, incl, 31);
-            if (run >= target) break;
+          for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+          }
+          const unsigned long long xa = s_above + incl - lm;  // mass of every larger value
+          __syncwarp();
+          if (xa < target && xa + mm[0] >= target) {  // the higher key of the word
+            s_kappa = 2u * static_cast<uint32_t>(word) + 1u;
+            s_above = xa;
+            s_c = cc[0];
+            s_each = mm[0] / cc[0];
+          } else if (xa + mm[0] < target && xa + lm >= target) {
+            s_kappa = 2u * static_cast<uint32_t>(word);
+            s_above = xa + mm[0];
+            s_c = cc[1];
+            s_each = mm[1] / cc[1];
           }
         }
         __syncthreads();

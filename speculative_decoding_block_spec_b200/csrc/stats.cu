@@ -360,7 +360,9 @@ int stats_grid(int dtype, bool vec, int64_t max_units, int64_t Vu) {
   int g;
   if (dtype == 0) g = vec ? occupancy_of<0, true>() : occupancy_of<0, false>();
   else g = vec ? occupancy_of<1, true>() : occupancy_of<1, false>();
-  const int64_t need = (max_units + kThreads - 1) / kThreads;  // at least one unit per thread
+  // at least one unit per thread, and up to one block per row: a small window's rows are then streamed in
+  // parallel rather than one after another by a single block
+  const int64_t need = std::max<int64_t>((max_units + kThreads - 1) / kThreads, (max_units + Vu - 1) / Vu);
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(g, need)));
 }
 

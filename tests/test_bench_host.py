@@ -44,7 +44,7 @@ def test_stats_kernel_choice_mirrors_the_library():
 def test_headline_is_the_largest_workload_and_extras_follow():
     a = bench.parse_args([])
     assert a.workload == 5 and synth.WORKLOADS[a.workload].name == "stress B64 L16 V151936 K4 bf16 budget544"
-    assert a.extra_ids == [2, 3, 4]
+    assert a.extra_ids == [1, 2, 3, 4]
     assert bench.parse_args(["--extras", ""]).extra_ids == []
     assert bench.parse_args(["--workload", "3", "--extras", "2,3"]).extra_ids == [2]
 
