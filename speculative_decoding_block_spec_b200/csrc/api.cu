@@ -226,9 +226,6 @@ int launch_nucleus_stage(const void* target, const int32_t* row_off, const void*
   char* w = static_cast<char*>(ws);
   NucleusArgs a = {};
   a.rs = verify_walk(target, row_off, draft, K, tokens, vlen, B, L, V, reinterpret_cast<float*>(w + lay.xg), true);
-  a.part = reinterpret_cast<const float2*>(w + lay.rpart);
-  a.G = stats_grid_of(dtype, vec, B, L, K, V, true);
-  a.Vu = units_per_row(V, dtype, vec);
   a.V = V;
   a.k = static_cast<float>(1.4426950408889634 / static_cast<double>(T));
   a.top_p = static_cast<double>(top_p);
@@ -286,8 +283,10 @@ int launch_accept_stage(const void* target, const int32_t* row_off, const void* 
   return map_cuda(launch_accept_sample(a, dtype, vec_term, st));
 }
 
-// top_p >= 1: unfiltered (two stages); below 1: statistics with bonus rows,
-// the nucleus kernel, then the filtered accept / sample stage.
+// top_p >= 1: unfiltered (two stages); below 1: the nucleus kernel (which
+// also finds every row's maximum and the drafted-token logits, in place of
+// the statistics stage) over the window with bonus rows, then the filtered
+// accept / sample stage.
 int verify_common(const void* target, const int32_t* row_off, const void* draft, const float* mix_w, int K,
                   int dtype, const int32_t* tokens, const int32_t* vlen, const float* u, const float* g, int B,
                   int L, int64_t V, float T, int32_t* accept_len, int32_t* out_tokens, void* ws, size_t ws_bytes,
@@ -297,12 +296,9 @@ int verify_common(const void* target, const int32_t* row_off, const void* draft,
   int e = verify_check(target, row_off, draft, mix_w, K, dtype, tokens, vlen, u, g, B, L, V, T, accept_len,
                        out_tokens, ws, ws_bytes, true, topp);
   if (e) return e;
-  e = launch_stats_stage(target, row_off, draft, K, dtype, tokens, vlen, B, L, V, T, ws, st, topp);
+  e = topp ? launch_nucleus_stage(target, row_off, draft, K, dtype, tokens, vlen, B, L, V, T, top_p, ws, st)
+           : launch_stats_stage(target, row_off, draft, K, dtype, tokens, vlen, B, L, V, T, ws, st);
   if (e) return e;
-  if (topp) {
-    e = launch_nucleus_stage(target, row_off, draft, K, dtype, tokens, vlen, B, L, V, T, top_p, ws, st);
-    if (e) return e;
-  }
   return launch_accept_stage(target, row_off, draft, mix_w, K, dtype, tokens, vlen, u, g, B, L, V, T, accept_len,
                              out_tokens, ws, st, topp);
 }

@@ -35,7 +35,10 @@
 
 namespace specv {
 
-constexpr int kDvlThreads = 1024;
+#ifndef SPECV_DVL_THREADS
+#define SPECV_DVL_THREADS 1024
+#endif
+constexpr int kDvlThreads = SPECV_DVL_THREADS;  // one block; 256 ... 1024 threads
 constexpr int kDvlWarps = kDvlThreads / 32;
 constexpr int kDvlMaxL = 32;  // SPEC_MAX_L
 

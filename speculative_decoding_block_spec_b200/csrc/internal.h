@@ -59,10 +59,7 @@ struct VerifyArgs {
 
 // The top-p nucleus kernel's inputs and outputs (one entry per walk row).
 struct NucleusArgs {
-  RowSpace rs;              // the verify walk, bonus rows included
-  const float2* part;       // row-statistics partials of that walk
-  int G;                    // row-statistics grid size
-  int64_t Vu;               // row-statistics units per row
+  RowSpace rs;              // the verify walk, bonus rows included; xg receives the drafted-token logits
   int64_t V;
   float k;                  // log2(e) / T
   double top_p;

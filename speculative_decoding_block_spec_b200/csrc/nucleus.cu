@@ -1,4 +1,5 @@
-// Top-p (nucleus) cut of every row of the verify window.
+// Top-p (nucleus) filtering of every row of the verify window, and the row
+// statistics the filtered verification needs.
 //
 // Target sampling with a temperature and a top-p filter, target
 // probabilities taken under the same sampling filter ("DBLAST: Dependent
@@ -14,29 +15,28 @@
 // last member; token v is kept iff x_v > x_c, or x_v == x_c and v <= v_c.
 //
 // k_nucleus, one row at a time per block (one block per SM, rows strided over
-// the grid):
-//  1. the row's maximum m from the statistics partials;
-//  2. bf16 rows: one pass counts the tokens of every bf16 value (65,536
-//     16-bit counters packed two to a 32-bit word in shared memory, native
-//     integer atomics, no exponential per token); then the warps walk the
-//     values from the largest down, each value's mass being its count times
-//     2^((x - m) k) in fixed point (scaled by 2^42, rounded), and find the
-//     value whose mass carries the running total across top_p * total.
-//     Sums are exact integers, so the cut does not depend on the order of
-//     any addition. A row whose counters could have overflowed (their total
-//     is not V) takes the radix path instead;
-//     fp32 rows: a radix descent over 32-bit order keys of the logits, per
-//     digit a shared-memory histogram of the fixed-point mass of the tokens
-//     that match the key prefix found so far (64-bit integer atomics) and a
-//     descending scan for the crossing digit: bits 31..20, 19..8, 7..0 (the
-//     last digit also counts tokens);
-//  3. at the cut value, the number n of its tokens needed to reach top_p;
-//     if not all of them are needed, the n-th such token in index order is
-//     found with a warp-ordered count (the tie cut);
-//  4. outputs: m, the log of the nucleus mass sum_{v kept} 2^((x_v - m) k)
-//     (the filtered rows' normaliser), the cut key and the cut token.
-// The counting pass streams the row from HBM; the tie cut re-reads it from
-// L2.
+// the grid), in place of the statistics kernel when rows are filtered:
+//  bf16 rows: one HBM pass counts the tokens of every bf16 bit pattern
+//    (65,536 16-bit counters packed two to a 32-bit word in shared memory,
+//    native integer atomics; -0 counted as +0) and records the drafted
+//    token's logit. Everything else follows from the counts: the row
+//    maximum m is the largest value present (a NaN or +inf present, or only
+//    -inf, marks the row non-finite); the warps walk the values from the
+//    largest down, each value's mass being its count times round(2^((x - m)
+//    k) 2^42), in exact integers: the total is the normaliser, and the value
+//    whose mass carries the running total across top_p * total is the cut.
+//    A row whose counters could have wrapped (their total is not V) takes
+//    the fp32 route below.
+//  fp32 rows: a pass for the maximum and the drafted token's logit, then a
+//    radix descent over 32-bit order keys: per digit (bits 31..20, 19..8,
+//    7..0) the fixed-point mass of the tokens matching the prefix found so
+//    far, with 64-bit integer atomics, and a descending scan for the digit
+//    where the running mass crosses top_p * total.
+//  Then the tokens of the cut value needed, n; if not all of them, the n-th
+//  in index order is found with a warp-ordered count (the tie cut), which
+//  re-reads the row from L2. Outputs per row: m, the log of the nucleus mass
+//  sum_{v kept} 2^((x_v - m) k) (the filtered normaliser), the cut key, the
+//  cut token and the drafted token's logit.
 #include <algorithm>
 
 #include "common.cuh"
@@ -234,8 +234,9 @@ __device__ __forceinline__ int64_t nth_equal(const char* row, int64_t V, uint32_
   return *s_v;
 }
 
-// Order key of a bf16 logit from its 16 bits (as order_key of the widened
-// value, shifted down 16), and the value of a key.
+// Order key of a bf16 logit from its 16 bits (order_key of the widened
+// value, shifted down 16), the value of a key, and the widened value's
+// 32-bit order key (its low half is fixed by the sign).
 __device__ __forceinline__ uint32_t order_key16(uint32_t h) {
   h &= 0xFFFFu;
   if (h == 0x8000u) h = 0u;
@@ -245,69 +246,110 @@ __device__ __forceinline__ float key16_value(uint32_t key) {
   const uint32_t h = (key & 0x8000u) ? (key & 0x7FFFu) : (~key & 0xFFFFu);
   return __uint_as_float(h << 16);
 }
-// The widened value's 32-bit order key: its low half is fixed by the sign.
 __device__ __forceinline__ uint32_t key16_to_key32(uint32_t key) {
   return (key << 16) | ((key & 0x8000u) ? 0u : 0xFFFFu);
 }
 
-// Order keys of the two bf16 values packed in a 32-bit word (each half as
-// order_key16 of its half): negative h -> ~h, non-negative h -> h | 0x8000,
-// and -0 takes the key of +0.
-__device__ __forceinline__ uint32_t order_keys2(uint32_t w) {
-  const uint32_t neg = ((w >> 15) & 0x00010001u) * 0x7FFFu;  // 0x7FFF in each negative half
-  return (w ^ (neg | 0x80008000u)) ^ __vcmpeq2(w, 0x80008000u);
-}
+// bf16 counters are indexed by bit pattern: pattern h in half h & 1 of word
+// h >> 1. In key order (descending value), key word kw (keys 2kw+1, 2kw)
+// lives in pattern word kw - 16384 for kw >= 16384 (non-negative values, the
+// higher key in the high half) and in pattern word 32767 - kw below (negative
+// values, the higher key in the low half).
+__device__ __forceinline__ int pattern_word(int kw) { return kw >= 16384 ? kw - 16384 : 32767 - kw; }
 
-// bf16: count the tokens of every value (the counter of key v is half v & 1
-// of word v >> 1: the low half for even keys).
+// Count the tokens of every bit pattern of a bf16 row (-0 as +0); the thread
+// that loads token `tok` (-1: none) returns its pattern in *tokbits.
 template <bool VEC>
-__device__ __forceinline__ void count_values(const char* row, int64_t V, uint32_t* cnt) {
+__device__ __forceinline__ void count_patterns(const char* row, int64_t V, uint32_t* cnt, int tok, uint32_t* tokbits) {
   if constexpr (VEC) {
     constexpr int U = 4;
-    const int64_t Vu = V / 8;
-    for (int64_t u0 = threadIdx.x; u0 < Vu; u0 += U * kNucThreads) {
+    const int Vu = static_cast<int>(V / 8);
+    for (int u0 = threadIdx.x; u0 < Vu; u0 += U * kNucThreads) {
       uint4 w[U];
 #pragma unroll
       for (int h = 0; h < U; ++h) {
-        const int64_t u = u0 + static_cast<int64_t>(h) * kNucThreads;
+        const int u = u0 + h * kNucThreads;
         w[h] = u < Vu ? ldg16(reinterpret_cast<const uint4*>(row) + u) : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
       for (int h = 0; h < U; ++h) {
-        if (u0 + static_cast<int64_t>(h) * kNucThreads >= Vu) break;
-        const uint32_t ws[4] = {w[h].x, w[h].y, w[h].z, w[h].w};
+        const int u = u0 + h * kNucThreads;
+        if (u >= Vu) break;
+        uint32_t ws[4] = {w[h].x, w[h].y, w[h].z, w[h].w};
+        if ((tok >> 3) == u) *tokbits = (ws[(tok & 7) >> 1] >> (16 * (tok & 1))) & 0xFFFFu;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const uint32_t key = order_keys2(ws[c]);
-          atomicAdd(&cnt[(key >> 1) & 0x7FFFu], 1u << ((key & 1u) << 4));
-          atomicAdd(&cnt[key >> 17], 1u << (((key >> 16) & 1u) << 4));
+          const uint32_t x = ws[c] ^ (__vcmpeq2(ws[c], 0x80008000u) & 0x80008000u);  // -0 -> +0
+          atomicAdd(&cnt[(x >> 1) & 0x7FFFu], 1u << ((x & 1u) << 4));
+          atomicAdd(&cnt[x >> 17], 1u << (((x >> 16) & 1u) << 4));
         }
       }
     }
   } else {
     const unsigned short* r16 = reinterpret_cast<const unsigned short*>(row);
     for (int64_t v = threadIdx.x; v < V; v += kNucThreads) {
-      const uint32_t key = order_key16(__ldg(r16 + v));
-      atomicAdd(&cnt[key >> 1], (key & 1u) ? 0x10000u : 1u);
+      uint32_t x = __ldg(r16 + v);
+      if (v == tok) *tokbits = x;
+      if (x == 0x8000u) x = 0u;
+      atomicAdd(&cnt[x >> 1], 1u << ((x & 1u) << 4));
     }
   }
 }
 
-// Tokens and fixed-point mass of the two keys of counter word `word`
-// (higher key first).
-__device__ __forceinline__ void word_mass(const uint32_t* cnt, int word, float m, float k, uint32_t (&c)[2],
-                                          unsigned long long (&mass)[2]) {
-  const uint32_t wv = cnt[word];
-  c[0] = wv >> 16;       // key 2 word + 1
-  c[1] = wv & 0xFFFFu;   // key 2 word
+// Counts of the two keys of key word kw, the higher key first.
+__device__ __forceinline__ void kword_counts(const uint32_t* cnt, int kw, uint32_t (&c)[2]) {
+  const uint32_t wv = cnt[pattern_word(kw)];
+  const uint32_t lo = wv & 0xFFFFu, hi = wv >> 16;
+  c[0] = kw >= 16384 ? hi : lo;
+  c[1] = kw >= 16384 ? lo : hi;
+}
+
+// ... and their fixed-point masses count * round(2^((x - m) k) 2^kFix).
+__device__ __forceinline__ void kword_mass(const uint32_t* cnt, int kw, float m, float k, uint32_t (&c)[2],
+                                           unsigned long long (&mass)[2]) {
+  kword_counts(cnt, kw, c);
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     mass[t] = 0ull;
     if (c[t]) {
-      const uint32_t key = 2u * static_cast<uint32_t>(word) + 1u - t;
+      const uint32_t key = 2u * static_cast<uint32_t>(kw) + 1u - t;
       mass[t] = static_cast<unsigned long long>(c[t]) * to_fixed(ex2((key16_value(key) - m) * k));
     }
   }
+}
+
+// fp32 rows, and bf16 rows whose counters wrapped: the row maximum, whether
+// the row holds a NaN, and the drafted token's logit (the thread that loads
+// it). Called by the whole block; the results are in shared memory.
+template <int DT, bool VEC>
+__device__ __forceinline__ void max_pass(const char* row, int64_t V, int tok, float* s_wmax, int* s_bad, float* s_xg,
+                                         float& m, bool& bad) {
+  constexpr int E = VEC ? Elem<DT>::kPerVec : 1;
+  const int64_t Vu = V / E;
+  float mx = -INFINITY;
+  bool nan = false;
+  for (int64_t u = threadIdx.x; u < Vu; u += kNucThreads) {
+    float x[E];
+    if constexpr (VEC) Elem<DT>::unpack(ldg16(reinterpret_cast<const uint4*>(row) + u), x);
+    else x[0] = Elem<DT>::at(row, u);
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      nan |= x[e] != x[e];
+      mx = fmaxf(mx, x[e]);
+      if (u * E + e == tok) *s_xg = x[e];
+    }
+  }
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  nan = __any_sync(0xffffffffu, nan);
+  if (lane == 0) s_wmax[w] = mx;
+  if (nan && lane == 0) *s_bad = 1;
+  __syncthreads();
+  m = -INFINITY;
+  for (int q = 0; q < kNucWarps; ++q) m = fmaxf(m, s_wmax[q]);
+  bad = *s_bad != 0 || !isfinite(m);
+  __syncthreads();
 }
 
 // Radix descent (fp32 rows, and bf16 rows whose counters could have
@@ -373,8 +415,8 @@ __device__ __forceinline__ void radix_cut(const char* row, int64_t V, float m, f
 
 template <int DT, bool VEC>
 __global__ void __launch_bounds__(kNucThreads, 1) k_nucleus(NucleusArgs a) {
-  // dynamic shared memory: a 128 KiB region (bf16 value counters, or the
-  // radix path's 4096 64-bit bins), then the walk (rowoff[B + 1], base[B])
+  // dynamic shared memory: a 128 KiB region (bf16 counters, or the radix
+  // path's 4096 64-bit bins), then the walk (rowoff[B + 1], base[B])
   extern __shared__ unsigned long long nuc_smem[];
   uint32_t* cnt = reinterpret_cast<uint32_t*>(nuc_smem);
   unsigned long long* hist = nuc_smem;
@@ -385,9 +427,12 @@ __global__ void __launch_bounds__(kNucThreads, 1) k_nucleus(NucleusArgs a) {
   __shared__ unsigned s_wc[kNucWarps];
   __shared__ unsigned long long s_step[kNucThreads];  // bf16: mass of each 32-word step, descending keys
   __shared__ unsigned s_wtok[kNucWarps];
-  __shared__ int s_sel;
-  __shared__ float s_m;
+  __shared__ int s_wkey[kNucWarps];
+  __shared__ float s_wmax[kNucWarps];
+  __shared__ int s_sel, s_bad, s_tok;
   __shared__ const char* s_row;
+  __shared__ uint32_t s_tokbits;
+  __shared__ float s_xg;
   __shared__ int s_d;
   __shared__ unsigned long long s_above, s_each;
   __shared__ unsigned s_c;
@@ -398,41 +443,23 @@ __global__ void __launch_bounds__(kNucThreads, 1) k_nucleus(NucleusArgs a) {
   const RowSpace& rs = a.rs;
   const Walk w{walk_smem, walk_smem + rs.B + 1};
   const int64_t nrows = build_walk<kNucThreads>(rs, walk_smem, s_itmp);
-  const int64_t N = nrows * a.Vu;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   for (int64_t r = blockIdx.x; r < nrows; r += gridDim.x) {
-    if (wid == 0) {  // the row maximum: the lanes load its partials in parallel (any order: a maximum)
-      const int64_t c0 = split_owner(r * a.Vu, N, a.G), c1 = split_owner((r + 1) * a.Vu - 1, N, a.G);
-      float mx = -INFINITY;
-      bool bad = false;
-      for (int64_t c = c0 + lane; c <= c1; c += 32) {
-        if (split_start(c + 1, N, a.G) == split_start(c, N, a.G)) continue;  // empty share: no partial
-        const float2 pr = __ldcg(a.part + c + r);
-        bad |= (pr.x != pr.x) || !isfinite(pr.y);
-        mx = fmaxf(mx, pr.x);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      bad = __any_sync(0xffffffffu, bad);
-      if (lane == 0) {
-        s_m = (!bad && isfinite(mx)) ? mx : NAN;
-        const int32_t* tokp;
-        s_row = locate<DT>(rs, w, r, tokp);
-      }
+    if (tid == 0) {
+      const int32_t* tokp;
+      s_row = locate<DT>(rs, w, r, tokp);
+      int tok = load_token(tokp);
+      if (tok >= a.V) tok = -1;  // out of range: flagged by the sampling kernel, nothing to record
+      s_tok = tok;
+      s_bad = 0;
+      s_tokbits = 0u;
+      s_xg = 0.f;
     }
     __syncthreads();
-    const float m = s_m;
     const char* row = s_row;
-    if (!(m == m)) {  // a non-finite row: the sampling kernel flags the request
-      if (tid == 0) {
-        a.row_m[r] = NAN;
-        a.row_lf[r] = NAN;
-        a.cut_key[r] = 0u;
-        a.cut_v[r] = static_cast<int32_t>(a.V - 1);
-      }
-      __syncthreads();
-      continue;
-    }
+    const int tok = s_tok;
+    float m = 0.f;
+    bool bad = false;
     unsigned long long whole = 0, target = 0, above = 0, each = 1;
     unsigned c = 0;
     uint32_t kappa = 0;
@@ -440,41 +467,68 @@ __global__ void __launch_bounds__(kNucThreads, 1) k_nucleus(NucleusArgs a) {
     if constexpr (DT == 1) {
       for (int i = tid; i < kValueWords / 4; i += kNucThreads) reinterpret_cast<uint4*>(cnt)[i] = make_uint4(0, 0, 0, 0);
       __syncthreads();
-      count_values<VEC>(row, a.V, cnt);
+      count_patterns<VEC>(row, a.V, cnt, tok, &s_tokbits);
       __syncthreads();
-      // step t = 32 wid + st covers counter words 32767 - 32 t down to 32767 - 32 t - 31 (keys descending),
-      // one word per lane; first the mass of every step, then a block scan over the 1024 steps, then the
-      // one step that holds the crossing
-      unsigned wt = 0;
+      // the largest value present, and whether a NaN or +inf is present (patterns 0x7F80.. and 0xFF81..)
+      int kmax = -1;
+      unsigned ntok = 0;
       for (int st = 0; st < 32; ++st) {
-        const int t = 32 * wid + st;
+        const int kw = kValueWords - 1 - 32 * (32 * wid + st) - lane;  // descending key words
         uint32_t cc[2];
-        unsigned long long mm[2];
-        word_mass(cnt, kValueWords - 1 - 32 * t - lane, m, a.k, cc, mm);
-        unsigned long long sm = mm[0] + mm[1];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
-        if (lane == 0) s_step[t] = sm;
-        wt += cc[0] + cc[1];
+        kword_counts(cnt, kw, cc);
+        ntok += cc[0] + cc[1];
+        if (cc[1]) kmax = max(kmax, 2 * kw);
+        if (cc[0]) kmax = max(kmax, 2 * kw + 1);
+        const int rw = pattern_word(kw);  // patterns 2rw, 2rw+1
+        const uint32_t p0 = 2u * rw, wv = cnt[rw];
+        const bool nonfin = ((wv & 0xFFFFu) && ((p0 & 0x7FFFu) >= 0x7F80u) && p0 != 0xFF80u) ||
+                            ((wv >> 16) && (((p0 + 1u) & 0x7FFFu) >= 0x7F80u));
+        if (nonfin) s_bad = 1;
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) wt += __shfl_xor_sync(0xffffffffu, wt, o);
-      if (lane == 0) s_wtok[wid] = wt;
-      if (tid == 0) {
-        s_c = 0u;
-        s_sel = 0;
+      for (int o = 16; o > 0; o >>= 1) {
+        kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+        ntok += __shfl_xor_sync(0xffffffffu, ntok, o);
+      }
+      if (lane == 0) {
+        s_wkey[wid] = kmax;
+        s_wtok[wid] = ntok;
       }
       __syncthreads();
-      const unsigned long long mine = s_step[tid];
-      const unsigned long long ex = block_scan_u64(mine, s_tmp);
-      if (tid == kNucThreads - 1) s_above = ex + mine;  // the whole mass
+      int kmx = -1;
       unsigned tokens = 0;
-      for (int q = 0; q < kNucWarps; ++q) tokens += s_wtok[q];
-      __syncthreads();
-      whole = s_above;
+      for (int q = 0; q < kNucWarps; ++q) {
+        kmx = max(kmx, s_wkey[q]);
+        tokens += s_wtok[q];
+      }
+      m = kmx >= 0 ? key16_value(static_cast<uint32_t>(kmx)) : NAN;
+      bad = s_bad != 0 || !isfinite(m);
+      if (tid == 0) s_xg = __uint_as_float(s_tokbits << 16);
       if (tokens != static_cast<unsigned>(a.V)) {
         radix = true;  // a value with more than 65,535 tokens wrapped its counter
-      } else {
+      } else if (!bad) {
+        // step t = 32 wid + st covers key words 32767 - 32 t down to 32767 - 32 t - 31, one per lane: the
+        // mass of every step, a block scan over the 1024 steps, then the one step that holds the crossing
+        for (int st = 0; st < 32; ++st) {
+          const int t = 32 * wid + st;
+          uint32_t cc[2];
+          unsigned long long mm[2];
+          kword_mass(cnt, kValueWords - 1 - 32 * t - lane, m, a.k, cc, mm);
+          unsigned long long sm = mm[0] + mm[1];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
+          if (lane == 0) s_step[t] = sm;
+        }
+        if (tid == 0) {
+          s_c = 0u;
+          s_sel = 0;
+        }
+        __syncthreads();
+        const unsigned long long mine = s_step[tid];
+        const unsigned long long ex = block_scan_u64(mine, s_tmp);
+        if (tid == kNucThreads - 1) s_above = ex + mine;  // the whole mass: the normaliser, scaled by 2^42
+        __syncthreads();
+        whole = s_above;
         target = static_cast<unsigned long long>(ceil(a.top_p * static_cast<double>(whole)));
         if (target < 1ull) target = 1ull;
         if (target > whole) target = whole;
@@ -484,11 +538,11 @@ __global__ void __launch_bounds__(kNucThreads, 1) k_nucleus(NucleusArgs a) {
           s_above = ex;
         }
         __syncthreads();
-        if (wid == 0) {  // walk the one step: a warp scan over its 32 words
-          const int word = kValueWords - 1 - 32 * s_sel - lane;
+        if (wid == 0) {  // walk the one step: a warp scan over its 32 key words
+          const int kw = kValueWords - 1 - 32 * s_sel - lane;
           uint32_t cc[2];
           unsigned long long mm[2];
-          word_mass(cnt, word, m, a.k, cc, mm);
+          kword_mass(cnt, kw, m, a.k, cc, mm);
           const unsigned long long lm = mm[0] + mm[1];
           unsigned long long incl = lm;
 #pragma unroll
@@ -499,12 +553,12 @@ __global__ void __launch_bounds__(kNucThreads, 1) k_nucleus(NucleusArgs a) {
           const unsigned long long xa = s_above + incl - lm;  // mass of every larger value
           __syncwarp();
           if (xa < target && xa + mm[0] >= target) {  // the higher key of the word
-            s_kappa = 2u * static_cast<uint32_t>(word) + 1u;
+            s_kappa = 2u * static_cast<uint32_t>(kw) + 1u;
             s_above = xa;
             s_c = cc[0];
             s_each = mm[0] / cc[0];
           } else if (xa + mm[0] < target && xa + lm >= target) {
-            s_kappa = 2u * static_cast<uint32_t>(word);
+            s_kappa = 2u * static_cast<uint32_t>(kw);
             s_above = xa + mm[0];
             s_c = cc[1];
             s_each = mm[1] / cc[1];
@@ -518,9 +572,23 @@ __global__ void __launch_bounds__(kNucThreads, 1) k_nucleus(NucleusArgs a) {
       }
       __syncthreads();
     }
-    if (radix)
-      radix_cut<DT, VEC>(row, a.V, m, a.k, a.top_p, hist, s_cnt, s_tmp, &s_d, &s_above, whole, target, above,
-                         kappa, c, each);
+    if (radix) {
+      max_pass<DT, VEC>(row, a.V, tok, s_wmax, &s_bad, &s_xg, m, bad);
+      if (!bad)
+        radix_cut<DT, VEC>(row, a.V, m, a.k, a.top_p, hist, s_cnt, s_tmp, &s_d, &s_above, whole, target, above,
+                           kappa, c, each);
+    }
+    if (bad) {  // a non-finite row: the sampling kernel flags the request
+      if (tid == 0) {
+        a.row_m[r] = NAN;
+        a.row_lf[r] = NAN;
+        a.cut_key[r] = 0u;
+        a.cut_v[r] = static_cast<int32_t>(a.V - 1);
+        if (tok >= 0) rs.xg[r] = s_xg;
+      }
+      __syncthreads();
+      continue;
+    }
     // tokens at the cut value: how many are needed, and which is the last
     const unsigned long long need = (target - above + each - 1) / each;
     const unsigned take = static_cast<unsigned>(need < c ? need : c);
@@ -532,6 +600,7 @@ __global__ void __launch_bounds__(kNucThreads, 1) k_nucleus(NucleusArgs a) {
       a.row_lf[r] = log(static_cast<double>(kept)) - kFix * 0.6931471805599453;
       a.cut_key[r] = kappa;
       a.cut_v[r] = static_cast<int32_t>(vcut);
+      if (tok >= 0) rs.xg[r] = s_xg;
     }
     __syncthreads();
   }

@@ -192,3 +192,73 @@ def test_workspace_reuse_and_status():
         acc, out = _verify(d, x, top_p, workspace=ws)
         check_verify(_cpu(acc), _cpu(out), ref)
     assert ws.status() & ~specv.DEV_NONFINITE == 0
+
+
+def test_dvl_packed_rows_with_top_p():
+    """Top-p on DVL-packed target rows (verify lengths and row offsets read on
+    the device): the bonus row of request b is packed row offsets[b] + l_b."""
+    x = synth.custom(B=16, L=12, V=32768, K=3, T=1.5, dtype="bf16", n_peaks=8, peak=4.0, draft_sigma=1.0,
+                     budget=16 * 13 // 2, seed=13, cid=670)
+    x = redraw_from_filtered(x, 0.95, seed=13)
+    w = x.w
+    rd = oracle.dvl_allocate(x.scores, w.budget)
+    packed_ref = oracle.pack(x.target, rd["verify_len"], rd["offsets"], w.budget)
+    ref = oracle.verify(packed_ref, x.draft, x.tokens, x.u, x.g, w.T, mix_w=x.mix_w, verify_len=rd["verify_len"],
+                        target_row_off=rd["offsets"][:w.B], n_threads=NT, diag=True, top_p=float(np.float32(0.95)))
+    d = to_torch(x)
+    packed = torch.zeros((w.budget, w.V), dtype=d["target"].dtype, device="cuda")
+    vl, off, _ = specv.dvl_allocate_pack(d["scores"], w.budget, dense_target=d["target"], packed_target=packed)
+    acc, out = specv.spec_verify_mixture_top_p(packed, d["draft"], d["mix_w"], d["tokens"], d["u"], d["g"], w.T,
+                                               0.95, verify_len=vl, target_row_off=off[:w.B])
+    check_verify(_cpu(acc), _cpu(out), ref, verify_len=rd["verify_len"])
+
+
+def test_graph_replay_with_top_p_across_allocations():
+    """One captured graph (DVL allocation, packing, filtered verification)
+    replayed with new survival scores and uniforms in the same buffers."""
+    B, L, V, K, T, top_p = 12, 10, 16384, 2, 1.3, 0.9
+    budget = B * (L + 1) // 2
+    x = redraw_from_filtered(synth.custom(B=B, L=L, V=V, K=K, T=T, dtype="bf16", n_peaks=6, peak=5.0,
+                                          draft_sigma=0.8, budget=budget, seed=14, cid=671), top_p, seed=14)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        d = to_torch(x)
+        packed = torch.zeros((budget, V), dtype=d["target"].dtype, device="cuda")
+        dvl_ws = specv.Workspace(specv.dvl_workspace_size(B))
+        ver_ws = specv.Workspace(specv.verify_top_p_workspace_size(B, L, K, V))
+        dvl_out = (torch.empty(B, dtype=torch.int32, device="cuda"), torch.empty(B + 1, dtype=torch.int32, device="cuda"),
+                   torch.empty(budget, dtype=torch.int32, device="cuda"))
+        ver_out = (torch.empty(B, dtype=torch.int32, device="cuda"),
+                   torch.empty((B, L + 1), dtype=torch.int32, device="cuda"))
+
+        def step():
+            vl, off, _ = specv.dvl_allocate_pack(d["scores"], budget, dense_target=d["target"], packed_target=packed,
+                                                 workspace=dvl_ws, out=dvl_out)
+            specv.spec_verify_mixture_top_p(packed, d["draft"], d["mix_w"], d["tokens"], d["u"], d["g"], T, top_p,
+                                            verify_len=vl, target_row_off=off[:B], workspace=ver_ws, out=ver_out)
+
+        step()
+        s.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=s):
+            step()
+        s.synchronize()
+    rng = np.random.default_rng(77)
+    seen = set()
+    for trial in range(4):
+        scores = -np.sort(-rng.beta(6.0 - trial, 2.0 + trial, size=(B, L)), axis=1).astype(np.float32)
+        u = rng.random((B, L), dtype=np.float32)
+        with torch.cuda.stream(s):
+            d["scores"].copy_(torch.from_numpy(scores))
+            d["u"].copy_(torch.from_numpy(u))
+            graph.replay()
+        s.synchronize()
+        rd = oracle.dvl_allocate(scores, budget)
+        np.testing.assert_array_equal(dvl_out[0].cpu().numpy(), rd["verify_len"])
+        pk = oracle.pack(x.target, rd["verify_len"], rd["offsets"], budget)
+        ref = oracle.verify(pk, x.draft, x.tokens, u, x.g, T, mix_w=x.mix_w, verify_len=rd["verify_len"],
+                            target_row_off=rd["offsets"][:B], n_threads=NT, diag=True, top_p=float(np.float32(top_p)))
+        check_verify(ver_out[0].cpu().numpy(), ver_out[1].cpu().numpy(), ref, verify_len=rd["verify_len"])
+        seen.add(tuple(rd["verify_len"]))
+    assert len(seen) > 1
+    assert ver_ws.status() & ~specv.DEV_NONFINITE == 0
