@@ -15,19 +15,23 @@
 //  1. one thread per request forms its products in fp64, left to right, and
 //     stores them as 64-bit keys whose unsigned order is the order of P
 //     (+0 and -0 are one key, as they compare equal);
-//  2. a radix select over the keys, 8-bit digits from the top, finds the
-//     (budget' - B)-th entry in the order (P desc, flat index asc): per digit
-//     a 256-bin histogram of the entries that still match the prefix (one
-//     shared atomic per distinct digit of a warp, grouped with
-//     __match_any_sync) and one warp's suffix scan over it; the descent
-//     stops at the first digit whose bin is taken whole;
-//  3. entries above the cut are selected, and of those equal to it the
-//     first ones by flat index (an exclusive scan over the equal-key flags,
-//     only when equal full keys straddle the cut);
-//  4. verify_len[b] = selected entries of row b; an exclusive scan of
+//  2. with every score in [0, 1] each row is already sorted in the global
+//     order (P desc, flat index asc), so for B*L <= 4096 the B rows are
+//     merged bottom-up: in each of ceil(log2 B) rounds every entry finds its
+//     rank in the partner list by binary search and moves to its merged
+//     position (one barrier per round); the selected entries are then the
+//     first budget' - B positions;
+//     otherwise (larger windows, or a flagged score that may unsort a row) a
+//     radix select over the keys, 8-bit digits from the top, finds the cut:
+//     per digit a 256-bin histogram of the entries that still match the
+//     prefix (one shared atomic per distinct digit of a warp, grouped with
+//     __match_any_sync) and one warp's suffix scan over it; the descent stops
+//     at the first digit whose bin is taken whole; entries above the cut are
+//     selected, and of those equal to it the first ones by flat index;
+//  3. verify_len[b] = selected entries of row b; an exclusive scan of
 //     verify_len + 1 gives the offsets, from which the slot map is filled.
-// O(B L) work per digit; k_dvl_pack then copies the selected dense target
-// rows into the fixed-address packed buffer.
+// k_dvl_pack then copies the selected dense target rows into the
+// fixed-address packed buffer.
 #include <algorithm>
 
 #include "common.cuh"
@@ -41,6 +45,7 @@ namespace specv {
 constexpr int kDvlThreads = SPECV_DVL_THREADS;  // one block; 256 ... 1024 threads
 constexpr int kDvlWarps = kDvlThreads / 32;
 constexpr int kDvlMaxL = 32;  // SPEC_MAX_L
+constexpr int kDvlMergeMax = 4096;  // B*L merged in shared memory (two key / index buffers)
 
 // Order-preserving key of a product: unsigned order of the key = numeric
 // order of P (negative values below +0; -0 maps to the key of +0; a NaN,
@@ -49,6 +54,27 @@ __device__ __forceinline__ unsigned long long p_key(double P) {
   if (P == 0.0) P = 0.0;
   const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(P));
   return (b >> 63) ? ~b : (b | (1ull << 63));
+}
+
+// offsets[0..B] from the scanned lengths `off` (off[B] = total), and the slot
+// map: slot s -> b * (L + 1) + (s - off[b]) for the request b holding it, -1
+// past the total. Called by the whole block.
+__device__ __forceinline__ void write_offsets_and_slots(const int* off, int B, int L, int budget, int total,
+                                                        int32_t* offsets, int32_t* slot_map) {
+  for (int r = threadIdx.x; r <= B; r += kDvlThreads) offsets[r] = off[r];
+  if (!slot_map) return;
+  for (int s = threadIdx.x; s < budget; s += kDvlThreads) {
+    int v = -1;
+    if (s < total) {
+      int lo = 0, hi = B - 1;  // last request with offset <= s
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (off[mid] <= s) lo = mid; else hi = mid - 1;
+      }
+      v = lo * (L + 1) + (s - off[lo]);
+    }
+    slot_map[s] = v;
+  }
 }
 
 __global__ void __launch_bounds__(kDvlThreads, 1) k_dvl_allocate(const float* __restrict__ scores, int B, int L,
@@ -87,6 +113,51 @@ __global__ void __launch_bounds__(kDvlThreads, 1) k_dvl_allocate(const float* __
 
   const int64_t cap = static_cast<int64_t>(B) * (L + 1);
   const int take = static_cast<int>(std::min<int64_t>(budget, cap)) - B;  // 0 <= take <= n
+  if (n <= kDvlMergeMax && s_flag == 0) {  // block-uniform: every row sorted, merge them
+    unsigned long long* kA = sKey;
+    unsigned long long* kB = sKey + n;
+    uint32_t* iA = reinterpret_cast<uint32_t*>(sKey + 2 * n);
+    uint32_t* iB = iA + n;
+    int* cnt = reinterpret_cast<int*>(iB + n);  // [B + 1]: selected entries per row, then lengths / offsets
+    for (int e = tid; e < n; e += kDvlThreads) iA[e] = static_cast<uint32_t>(e);
+    for (int r = tid; r <= B; r += kDvlThreads) cnt[r] = 0;
+    __syncthreads();
+    for (int W = L; W < n; W *= 2) {  // lists of W entries, merged in pairs
+      for (int e = tid; e < n; e += kDvlThreads) {
+        const int base = (e / (2 * W)) * (2 * W);
+        const int mid = min(base + W, n), end = min(base + 2 * W, n);
+        const unsigned long long ke = kA[e];
+        const uint32_t ie = iA[e];
+        // entries of the other list that precede (ke, ie) in the order (key desc, index asc) form a prefix
+        int lo = e < mid ? mid : base, hi = e < mid ? end : mid;
+        const int first = lo;
+        while (lo < hi) {
+          const int md = (lo + hi) >> 1;
+          const unsigned long long km = kA[md];
+          if (km > ke || (km == ke && iA[md] < ie)) lo = md + 1; else hi = md;
+        }
+        const int pos = base + (e < mid ? e - base : e - mid) + (lo - first);
+        kB[pos] = ke;
+        iB[pos] = ie;
+      }
+      __syncthreads();
+      unsigned long long* tk = kA; kA = kB; kB = tk;
+      uint32_t* ti = iA; iA = iB; iB = ti;
+    }
+    for (int q = tid; q < take; q += kDvlThreads) atomicAdd(&cnt[iA[q] / L], 1);  // the first take are selected
+    __syncthreads();
+    for (int r = tid; r < B; r += kDvlThreads) {
+      const int ell = cnt[r];
+      verify_len[r] = ell;
+      cnt[r] = ell + 1;
+    }
+    __syncthreads();
+    const int total = block_exclusive_scan<kDvlThreads>(cnt, B, s_tmp);
+    if (tid == 0) cnt[B] = total;
+    __syncthreads();
+    write_offsets_and_slots(cnt, B, L, budget, total, offsets, slot_map);
+    return;  // scores all in [0, 1]: no flag to raise
+  }
   // The cut: entries whose key, under `mask`, is above `prefix` are selected; of those equal to it under the
   // mask, all are selected when the bin holds exactly the k still wanted, else (equal full keys) the first k
   // by flat index. take == 0 selects nothing: no masked key exceeds the all-ones prefix.
@@ -166,21 +237,7 @@ __global__ void __launch_bounds__(kDvlThreads, 1) k_dvl_allocate(const float* __
   const int total = block_exclusive_scan<kDvlThreads>(lens, B, s_tmp);
   if (tid == 0) lens[B] = total;
   __syncthreads();
-  for (int r = tid; r <= B; r += kDvlThreads) offsets[r] = lens[r];
-  if (slot_map) {
-    for (int s = tid; s < budget; s += kDvlThreads) {
-      int v = -1;
-      if (s < total) {
-        int lo = 0, hi = B - 1;  // last request with offset <= s
-        while (lo < hi) {
-          const int mid = (lo + hi + 1) >> 1;
-          if (lens[mid] <= s) lo = mid; else hi = mid - 1;
-        }
-        v = lo * (L + 1) + (s - lens[lo]);
-      }
-      slot_map[s] = v;
-    }
-  }
+  write_offsets_and_slots(lens, B, L, budget, total, offsets, slot_map);
   if (tid == 0 && s_flag) atomicOr(status, s_flag);
 }
 
@@ -223,8 +280,12 @@ __global__ void __launch_bounds__(kThreads) k_dvl_pack(const char* __restrict__ 
 cudaError_t launch_dvl(const float* scores, int B, int L, int budget, int32_t* verify_len, int32_t* offsets,
                        int32_t* slot_map, int* status, cudaStream_t st) {
   const int64_t n = static_cast<int64_t>(B) * L;
-  const size_t smem = static_cast<size_t>(n) * (sizeof(unsigned long long) + sizeof(int)) +
-                      static_cast<size_t>(B + 1) * sizeof(int);
+  // radix path: keys + equal ranks + lengths; merge path (B*L <= kDvlMergeMax): two key and index buffers
+  const size_t radix = static_cast<size_t>(n) * (sizeof(unsigned long long) + sizeof(int)) +
+                       static_cast<size_t>(B + 1) * sizeof(int);
+  const size_t merge = static_cast<size_t>(n) * 2 * (sizeof(unsigned long long) + sizeof(uint32_t)) +
+                       static_cast<size_t>(B + 1) * sizeof(int);
+  const size_t smem = n <= kDvlMergeMax ? std::max(radix, merge) : radix;
   if (smem > 48 * 1024) {
     const cudaError_t e =
         cudaFuncSetAttribute(k_dvl_allocate, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));

@@ -378,24 +378,56 @@ __global__ void __launch_bounds__(kThreads, 3) k_accept_sample(VerifyArgs a, flo
             }
           }
         }
-        // exact scores of every thread's two candidates; the block's best is a lower bound on its maximum
-        double e1, e2;
-        residual_score2<DT, TP>(trow, grow, dbase, dstride, K, s_c, s_mm, k, s_tk, s_tv, w1, w2, e1, e2);
-        if (e1 > -INFINITY) best_merge(br, Best{e1, w1});
-        if (e2 > -INFINITY) best_merge(br, Best{e2, w2});
-        Best wb = br;
-        warp_best(wb);
-        if (lane == 0) s_best[tid >> 5] = wb;
-        __syncthreads();
-        double lb = -INFINITY;
+        // Round 1: the exact score of each warp's largest bound (8 tokens per block); their best is a
+        // lower bound lb on the block's maximum. If none of them has p > q, round 1b scores every
+        // thread's two candidates.
+        bool ev1 = false, ev2 = false;  // w1 / w2 of this thread already scored
+        float wt = t1;
+        int wl = lane;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) lb = fmax(lb, s_best[w].score);
-        __syncthreads();
+        for (int o = 16; o > 0; o >>= 1) {
+          const float ot = __shfl_xor_sync(0xffffffffu, wt, o);
+          const int ol = __shfl_xor_sync(0xffffffffu, wl, o);
+          if (ot > wt || (ot == wt && ol < wl)) {
+            wt = ot;
+            wl = ol;
+          }
+        }
+        if (lane == wl && w1 >= 0) {
+          double e1, unused;
+          residual_score2<DT, TP>(trow, grow, dbase, dstride, K, s_c, s_mm, k, s_tk, s_tv, w1, -1, e1, unused);
+          if (e1 > -INFINITY) best_merge(br, Best{e1, w1});
+          ev1 = true;
+        }
+        double lb = -INFINITY;
+        for (int round = 0; round < 2; ++round) {
+          Best wb = br;
+          warp_best(wb);
+          if (lane == 0) s_best[tid >> 5] = wb;
+          __syncthreads();
+#pragma unroll
+          for (int w = 0; w < kWarps; ++w) lb = fmax(lb, s_best[w].score);
+          __syncthreads();
+          if (lb > -INFINITY || round == 1) break;  // block-uniform
+          double e1, e2;  // round 1b
+          residual_score2<DT, TP>(trow, grow, dbase, dstride, K, s_c, s_mm, k, s_tk, s_tv, ev1 ? -1 : w1, w2, e1, e2);
+          if (e1 > -INFINITY) best_merge(br, Best{e1, w1});
+          if (e2 > -INFINITY) best_merge(br, Best{e2, w2});
+          ev1 = ev2 = true;
+        }
         if (lb > -INFINITY) {  // block-uniform
           stream = false;
-          // Pass 2 (the share again, from L2), only in threads where a token other than w1, w2 may
-          // reach lb: every such token is scored exactly.
+          // Round 2: every token whose bound reaches lb - slack is scored exactly: this thread's w1 and
+          // w2 if not yet scored, and, when its third bound reaches the cut too, every other token of
+          // its share (read again, from L2).
           const float cut = static_cast<float>(lb) - kPruneSlack;
+          const int q1 = (!ev1 && t1 >= cut) ? w1 : -1, q2 = (!ev2 && t2 >= cut) ? w2 : -1;
+          if (q1 >= 0 || q2 >= 0) {
+            double e1, e2;
+            residual_score2<DT, TP>(trow, grow, dbase, dstride, K, s_c, s_mm, k, s_tk, s_tv, q1, q2, e1, e2);
+            if (e1 > -INFINITY) best_merge(br, Best{e1, q1});
+            if (e2 > -INFINITY) best_merge(br, Best{e2, q2});
+          }
           if (t3 >= cut) {
             for (int64_t u = ua; u < u1; u += kThreads) {
               float xt[E], gv[E];
