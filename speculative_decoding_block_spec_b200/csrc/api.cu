@@ -117,11 +117,12 @@ int accept_slots(int dtype, bool vec, int K, bool topp) {
 
 // Verify workspace: persistent state first (zero between calls), then scratch.
 // The walk has B (K+1) L rows, plus one bonus row per request with top-p
-// filtering, whose nucleus kernel adds four per-row arrays.
+// filtering, whose nucleus kernels add five per-row arrays.
 struct VerifyLayout {
   size_t ticket, keys;     // persistent: per-request tickets [B], terminal keys [2B]
   size_t xg, rpart;        // scratch
-  size_t nm, nlf, nkey, nv;  // top-p scratch: row maxima, log nucleus masses, cut keys, cut tokens
+  size_t nm, nlf, nkey, nv;  // top-p scratch: row maxima, log nucleus masses, cut keys, cut tokens,
+  size_t nflag;              // and the rows the fast nucleus kernel hands to the exact one
   size_t total;
 };
 
@@ -138,13 +139,14 @@ VerifyLayout verify_layout(int B, int L, int K, int64_t V, bool topp = false) {
   l.xg = l.keys + align256(static_cast<size_t>(2 * B) * sizeof(unsigned long long));
   l.rpart = l.xg + align256(rows * sizeof(float));
   l.total = l.rpart + align256((static_cast<size_t>(kGMax) + rows) * sizeof(float2));
-  l.nm = l.nlf = l.nkey = l.nv = 0;
+  l.nm = l.nlf = l.nkey = l.nv = l.nflag = 0;
   if (topp) {
     l.nm = l.total;
     l.nlf = l.nm + align256(rows * sizeof(float));
     l.nkey = l.nlf + align256(rows * sizeof(double));
     l.nv = l.nkey + align256(rows * sizeof(uint32_t));
-    l.total = l.nv + align256(rows * sizeof(int32_t));
+    l.nflag = l.nv + align256(rows * sizeof(int32_t));
+    l.total = l.nflag + align256(rows * sizeof(int));
   }
   return l;
 }
@@ -233,6 +235,13 @@ int launch_nucleus_stage(const void* target, const int32_t* row_off, const void*
   a.row_lf = reinterpret_cast<double*>(w + lay.nlf);
   a.cut_key = reinterpret_cast<uint32_t*>(w + lay.nkey);
   a.cut_v = reinterpret_cast<int32_t*>(w + lay.nv);
+  // bf16 rows of 16-byte vectors: the windowed kernel first, the exact one for the rows it hands over
+  if (dtype == 1 && vec && V >= kNucFastMinV) {
+    a.flags = reinterpret_cast<int*>(w + lay.nflag);
+    const cudaError_t e = launch_nucleus_fast(a, st);
+    if (e != cudaSuccess) return map_cuda(e);
+    a.only = a.flags;
+  }
   return map_cuda(launch_nucleus(a, dtype, vec, st));
 }
 

@@ -67,6 +67,8 @@ struct NucleusArgs {
   double* row_lf;           // out: log of the nucleus mass sum_{v kept} 2^((x_v - m) k)
   uint32_t* cut_key;        // out: order key of the cut value
   int32_t* cut_v;           // out: cut token (tokens at the cut value with index <= cut_v are kept)
+  int* flags;               // fast path, out: 1 for a row it hands to the exact kernel, else 0
+  const int* only;          // exact kernel (nullable): process only the rows whose entry is non-zero
 };
 
 // Units of work per row: 16-byte vectors on the vector path, else elements.
@@ -85,6 +87,8 @@ cudaError_t launch_softmax_finalize(const void* logits, int dtype, bool vec, int
                                     float* row_lse, float* probs, cudaStream_t st);
 
 cudaError_t launch_nucleus(const NucleusArgs& a, int dtype, bool vec, cudaStream_t st);
+cudaError_t launch_nucleus_fast(const NucleusArgs& a, cudaStream_t st);  // bf16 rows of 16-byte vectors
+constexpr int64_t kNucFastMinV = 4096;  // smaller rows take the exact kernel alone
 
 cudaError_t launch_accept_sample(const VerifyArgs& a, int dtype, bool vec, cudaStream_t st);
 int accept_blocks_per_sm(int dtype, bool vec, int K, bool topp);

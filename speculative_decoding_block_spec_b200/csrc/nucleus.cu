@@ -64,31 +64,38 @@ __device__ __forceinline__ unsigned long long to_fixed(float q) {
   return static_cast<unsigned long long>((mant + (1u << (-sh - 1))) >> (-sh));
 }
 
-// Block-wide exclusive scan of one 64-bit value per thread (thread order);
-// `tmp` holds kNucWarps + 1 values. Returns the exclusive prefix.
-__device__ __forceinline__ unsigned long long block_scan_u64(unsigned long long v, unsigned long long* tmp) {
+// Block-wide exclusive scan of one value per thread (thread order), for a
+// block of NT threads; `tmp` holds NT / 32 + 1 values. Returns the exclusive
+// prefix.
+template <typename T, int NT>
+__device__ __forceinline__ T block_scan(T v, T* tmp) {
+  constexpr int NW = NT / 32;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  unsigned long long incl = v;
+  T incl = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const unsigned long long t = __shfl_up_sync(0xffffffffu, incl, o);
+    const T t = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += t;
   }
   if (lane == 31) tmp[w] = incl;
   __syncthreads();
   if (threadIdx.x == 0) {
-    unsigned long long run = 0;
-    for (int k = 0; k < kNucWarps; ++k) {
-      const unsigned long long t = tmp[k];
+    T run = 0;
+    for (int k = 0; k < NW; ++k) {
+      const T t = tmp[k];
       tmp[k] = run;
       run += t;
     }
-    tmp[kNucWarps] = run;
+    tmp[NW] = run;
   }
   __syncthreads();
-  const unsigned long long excl = tmp[w] + incl - v;
+  const T excl = tmp[w] + incl - v;
   __syncthreads();
   return excl;
+}
+
+__device__ __forceinline__ unsigned long long block_scan_u64(unsigned long long v, unsigned long long* tmp) {
+  return block_scan<unsigned long long, kNucThreads>(v, tmp);
 }
 
 // One digit of the descent: hist[d] += fixed mass of every token whose key
@@ -157,13 +164,13 @@ __device__ __forceinline__ void find_digit(const unsigned long long* hist, int n
 
 // Index (in row order) of the n-th token (1-based) whose key is kappa; the
 // row holds at least n of them. Called by the whole block.
-template <int DT, bool VEC>
+template <int DT, bool VEC, int NW = kNucWarps>
 __device__ __forceinline__ int64_t nth_equal(const char* row, int64_t V, uint32_t kappa, unsigned n, unsigned* s_wc,
                                              long long* s_v) {
   constexpr int E = VEC ? Elem<DT>::kPerVec : 1;
   const int64_t Vu = V / E;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int64_t cw = (Vu + kNucWarps - 1) / kNucWarps;  // units per warp, contiguous
+  const int64_t cw = (Vu + NW - 1) / NW;  // units per warp, contiguous
   const int64_t a = min(Vu, w * cw), b = min(Vu, a + cw);
   // bf16 vectors compare raw bit pairs: the raw bits of the cut value (and
   // those of -0 when the cut value is zero) in both halves of a word
@@ -445,6 +452,7 @@ __global__ void __launch_bounds__(kNucThreads, 1) k_nucleus(NucleusArgs a) {
   const int64_t nrows = build_walk<kNucThreads>(rs, walk_smem, s_itmp);
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   for (int64_t r = blockIdx.x; r < nrows; r += gridDim.x) {
+    if (a.only && !__ldcg(a.only + r)) continue;  // the fast path served this row (block-uniform)
     if (tid == 0) {
       const int32_t* tokp;
       s_row = locate<DT>(rs, w, r, tokp);
@@ -604,6 +612,425 @@ __global__ void __launch_bounds__(kNucThreads, 1) k_nucleus(NucleusArgs a) {
     }
     __syncthreads();
   }
+}
+
+// ---------------------------------------------------------------- fast path
+//
+// k_nucleus_fast, bf16 rows of 16-byte vectors: the cut is found inside a
+// narrow window of values chosen from a sample, so a token costs one
+// exponential and a few compares, and only the tokens inside the window are
+// counted; a row the window does not serve is handed to k_nucleus (flag 1).
+//  1. sample: 512 evenly spaced 16-byte units (4,096 logits); their maximum
+//     is the row's reference r (masses are 2^((x - r) k), relative to r);
+//  2. a histogram of the sample's masses over 4,096 bins of 16 consecutive
+//     16-bit order keys; scanning it from the top brackets the crossing of
+//     top_p: the bins between mass fractions top_p - delta and top_p + delta,
+//     delta four standard errors of the sample's estimate (effective size
+//     (sum q)^2 / sum q^2) plus 0.002, form the window, at most 1,024 keys
+//     (narrowed around the estimated crossing when wider), never reaching the
+//     patterns of infinities and NaNs;
+//  3. one HBM pass: every token adds its mass to the total (fp32 per 16-byte
+//     unit, fp64 per thread), tokens above the window also to the mass above,
+//     and tokens inside it are counted per value (shared reductions);
+//  4. the window's values, from the top, each with mass count * 2^((x - r) k)
+//     (exact in fp64): the value where the mass above plus the running sum
+//     reaches top_p * total is the cut. When the crossing lies above (below)
+//     the window, one more pass counts the 1,024 keys just above (below) it;
+//     when it misses again, or the row holds a NaN or an infinity, the row is
+//     flagged;
+//  5. the tie cut, as in k_nucleus.
+// Rows are never wrong for a poor sample, only handed over: every mass that
+// decides the cut is summed over the whole row.
+constexpr int kFastThreads = 256;
+constexpr int kFastWarps = kFastThreads / 32;
+constexpr int kSampleUnits = 2 * kFastThreads;
+constexpr int kSampleBins = 4096;  // 16 keys each
+constexpr int kWinKeys = 1024;
+constexpr int kFiniteKeyLo = 0x0080, kFiniteKeyHi = 0xFF7F;  // keys of -max finite and +max finite
+
+__device__ __forceinline__ unsigned long long pack_f2(float lo, float hi) {
+  unsigned long long v;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(lo), "f"(hi));
+  return v;
+}
+__device__ __forceinline__ void unpack_f2(unsigned long long v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long add_f2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long mul_f2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ void red_if(uint32_t addr, uint32_t v, uint32_t limit) {  // count at addr when v <= limit
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.le.u32 p, %1, %2;\n\t@p red.shared.add.u32 [%0], 1;\n\t}"
+               :: "r"(addr), "r"(v), "r"(limit) : "memory");
+}
+
+// One warp's share [ua, ub) (16-byte units) of a bf16 row for k_nucleus_fast:
+// the row's mass 2^((x - r) k) summed (fp32 per unit, two tokens at a time in
+// packed f32x2 arithmetic, fp64 across units), the part of it above the key
+// window [klo, khi], and a count per window key in this warp's counters
+// (shared address wcnt). The window index of a token comes from its bf16
+// bits h, by the window's place:
+//   MODE 1, window below zero (khi <= 0x7FFE): key = 0xFFFF - h for every
+//     negative value; every non-negative value (-0 too) lies above;
+//   MODE 2, window above zero (klo >= 0x8001): key = h + 0x8000 for every
+//     positive value; h sign-extended puts every negative pattern and both
+//     zeros below;
+//   MODE 0, any window: the 32-bit order key of x + 0 (so -0 counts as +0),
+//     f ^ ((f >> 31) | 0x80000000), whose top half is the 16-bit key.
+// A NaN lands above or below the window and its mass poisons the total.
+template <int MODE>
+__device__ __forceinline__ void window_unit(const uint4& v, unsigned long long nrr2, unsigned long long kk2, int klo,
+                                            int khi, uint32_t wcnt, double& tot, double& above) {
+  const int span = khi - klo;
+  const int c1 = 0xFFFF - klo, c2 = 0x8000 - klo;
+  const uint32_t klo32 = static_cast<uint32_t>(klo) << 16, khi32 = (static_cast<uint32_t>(khi) << 16) | 0xFFFFu;
+  const uint32_t ws[4] = {v.x, v.y, v.z, v.w};
+  unsigned long long ts2 = 0ull;
+  float as = 0.f;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint32_t f[2] = {ws[c] << 16, ws[c] & 0xFFFF0000u};
+    float e[2], q[2];
+    unpack_f2(mul_f2(add_f2(pack_f2(__uint_as_float(f[0]), __uint_as_float(f[1])), nrr2), kk2), e[0], e[1]);
+    q[0] = ex2(e[0]);
+    q[1] = ex2(e[1]);
+    ts2 = add_f2(ts2, pack_f2(q[0], q[1]));
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      if constexpr (MODE == 0) {
+        const uint32_t g = __float_as_uint(__uint_as_float(f[half]) + 0.f);
+        const uint32_t key32 = g ^ (static_cast<uint32_t>(static_cast<int32_t>(g) >> 31) | 0x80000000u);
+        if (key32 > khi32) as += q[half];
+        const uint32_t off = key32 - klo32;
+        red_if(wcnt + ((off >> 16) << 2), off, khi32 - klo32);
+      } else {
+        const int idx = MODE == 1 ? c1 - static_cast<int>(f[half] >> 16) : (static_cast<int32_t>(f[half]) >> 16) + c2;
+        if (idx > span) as += q[half];
+        red_if(wcnt + (static_cast<uint32_t>(idx) << 2), static_cast<uint32_t>(idx), static_cast<uint32_t>(span));
+      }
+    }
+  }
+  float t0, t1;
+  unpack_f2(ts2, t0, t1);
+  tot += static_cast<double>(t0 + t1);
+  above += static_cast<double>(as);
+}
+
+template <int MODE>
+__device__ __forceinline__ void window_stream(const char* row, int ua, int ub, int lane, float rr, float kk, int klo,
+                                              int khi, uint32_t wcnt, double& tot, double& above) {
+  const unsigned long long nrr2 = pack_f2(-rr, -rr), kk2 = pack_f2(kk, kk);
+  const uint4* src = reinterpret_cast<const uint4*>(row);
+  constexpr int U = 4;
+  int u0 = ua + lane;
+  for (; u0 + 32 * (U - 1) < ub; u0 += 32 * U) {  // whole groups: no bounds checks
+    uint4 wv[U];
+#pragma unroll
+    for (int h = 0; h < U; ++h) wv[h] = ldg16(src + u0 + 32 * h);
+#pragma unroll
+    for (int h = 0; h < U; ++h) window_unit<MODE>(wv[h], nrr2, kk2, klo, khi, wcnt, tot, above);
+  }
+  for (; u0 < ub; u0 += 32) window_unit<MODE>(ldg16(src + u0), nrr2, kk2, klo, khi, wcnt, tot, above);
+}
+
+__global__ void __launch_bounds__(kFastThreads, 4) k_nucleus_fast(NucleusArgs a) {
+  extern __shared__ int walk_smem[];  // rowoff[B + 1], base[B]
+  // one 32 KB area: the sample's bins (fp32), then the window's counters (one set per warp)
+  __shared__ __align__(16) uint32_t s_area[kFastWarps * kWinKeys];
+  float* const s_bm = reinterpret_cast<float*>(s_area);
+  __shared__ float s_ftmp[kFastWarps + 1];
+  __shared__ double s_dtmp[kFastWarps + 1];
+  __shared__ double s_red[2 * kFastWarps];
+  __shared__ float s_fred[2 * kFastWarps];
+  __shared__ int s_itmp[kFastWarps + 1];
+  __shared__ unsigned s_wc[kFastWarps];
+  __shared__ const char* s_row;
+  __shared__ int s_tok, s_bhi, s_blo, s_bst, s_klo, s_khi, s_kappa, s_wsel;
+  __shared__ float s_xg;
+  __shared__ double s_before, s_qk;
+  __shared__ unsigned s_ck, s_nth;
+  __shared__ long long s_v;
+  pdl_wait();
+  pdl_trigger();
+  const RowSpace& rs = a.rs;
+  const Walk w{walk_smem, walk_smem + rs.B + 1};
+  const int64_t nrows = build_walk<kFastThreads>(rs, walk_smem, s_itmp);
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int Vu = static_cast<int>(a.V / 8);
+  const float kk = a.k;
+  for (int64_t r = blockIdx.x; r < nrows; r += gridDim.x) {
+    if (tid == 0) {
+      const int32_t* tokp;
+      s_row = locate<1>(rs, w, r, tokp);
+      int tok = load_token(tokp);
+      if (tok >= a.V) tok = -1;
+      s_tok = tok;
+      s_xg = tok >= 0 ? __uint_as_float(static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short*>(s_row) + tok)) << 16)
+                      : 0.f;
+      s_bhi = s_blo = s_bst = -1;
+    }
+    for (int i = tid; i < kSampleBins; i += kFastThreads) s_bm[i] = 0.f;
+    __syncthreads();
+    const char* row = s_row;
+    const int tok = s_tok;
+    // 1. the sample (two units per thread, in registers) and its maximum
+    float xs[16];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int j = tid + h * kFastThreads;
+      const int u = static_cast<int>(((2ll * j + 1) * Vu) / (2 * kSampleUnits));
+      float x8[8];
+      Elem<1>::unpack(ldg16(reinterpret_cast<const uint4*>(row) + u), x8);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) xs[8 * h + e] = x8[e];
+    }
+    float lm = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) lm = fmaxf(lm, xs[e]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, o));
+    if (lane == 0) s_fred[wid] = lm;
+    __syncthreads();
+    float rr = -INFINITY;
+    for (int q = 0; q < kFastWarps; ++q) rr = fmaxf(rr, s_fred[q]);
+    const bool rok = isfinite(rr);
+    // 2. the sample's masses over the bins
+    float sq = 0.f, sq2 = 0.f;
+    if (rok) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float q = ex2((xs[e] - rr) * kk);
+        if (q == q) {
+          atomicAdd(&s_bm[order_key16(__float_as_uint(xs[e]) >> 16) >> 4], q);
+          sq += q;
+          sq2 += q * q;
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      sq += __shfl_xor_sync(0xffffffffu, sq, o);
+      sq2 += __shfl_xor_sync(0xffffffffu, sq2, o);
+    }
+    __syncthreads();  // every thread has read the maxima from s_fred
+    if (lane == 0) {
+      s_fred[wid] = sq;
+      s_fred[kFastWarps + wid] = sq2;
+    }
+    __syncthreads();
+    float stot = 0.f, stot2 = 0.f;
+    for (int q = 0; q < kFastWarps; ++q) {
+      stot += s_fred[q];
+      stot2 += s_fred[kFastWarps + q];
+    }
+    const float tp = static_cast<float>(a.top_p);
+    const float neff = stot2 > 0.f ? stot * stot / stot2 : 1.f;
+    const float delta = 4.f * sqrtf(tp * (1.f - tp) / fmaxf(neff, 1.f)) + 0.002f;
+    const float lo_t = (tp - delta) * stot, hi_t = (tp + delta) * stot, st_t = tp * stot;
+    {  // thread t: bins 4095 - 16t down to 4080 - 16t; the first bins (from the top) past each threshold
+      float c[16], sum = 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        c[j] = s_bm[kSampleBins - 1 - 16 * tid - j];
+        sum += c[j];
+      }
+      float run = block_scan<float, kFastThreads>(sum, s_ftmp);
+      int bhi = -1, blo = -1, bst = -1;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        run += c[j];
+        const int b = kSampleBins - 1 - 16 * tid - j;
+        if (run > lo_t && bhi < 0) bhi = b;
+        if (run >= hi_t && blo < 0) blo = b;
+        if (run >= st_t && bst < 0) bst = b;
+      }
+      if (bhi >= 0) atomicMax(&s_bhi, bhi);
+      if (blo >= 0) atomicMax(&s_blo, blo);
+      if (bst >= 0) atomicMax(&s_bst, bst);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int bhi = s_bhi, blo = s_blo;
+      if (blo < 0) blo = 0;  // top_p + delta is past the sample's mass: down to the lowest finite key
+      if (bhi - blo + 1 > kWinKeys / 16) {  // too wide: around the estimated crossing
+        bhi = min(bhi, s_bst + kWinKeys / 32 - 1);
+        blo = max(blo, bhi - kWinKeys / 16 + 1);
+      }
+      const int klo = max(16 * blo, kFiniteKeyLo), khi = min(16 * bhi + 15, kFiniteKeyHi);
+      s_klo = klo;
+      s_khi = (!rok || bhi < 0 || khi < klo) ? -1 : khi;  // -1: no usable window
+    }
+    __syncthreads();
+    if (s_khi < 0) {  // the exact kernel takes the row
+      if (tid == 0) a.flags[r] = 1;
+      __syncthreads();
+      continue;
+    }
+    // 3./4. up to two passes; every decision below is block-uniform. Warp w streams units [w cw, (w+1) cw)
+    //    and counts its window keys in its own counters, so the tie search reads one chunk again, not the
+    //    row
+    const int cw = (Vu + kFastWarps - 1) / kFastWarps;
+    const int ua = min(Vu, wid * cw), ub = min(Vu, ua + cw);
+    const uint32_t wcnt = static_cast<uint32_t>(__cvta_generic_to_shared(s_area + wid * kWinKeys));
+    bool done = false, hand = false;
+    double target = 0.0;
+    for (int pass = 0; pass < 2 && !done && !hand; ++pass) {
+      const int klo = s_klo, khi = s_khi;
+      __syncthreads();  // every thread has read the window and, in the first pass, the sample's bins
+      for (int i = tid; i < kFastWarps * kWinKeys; i += kFastThreads) s_area[i] = 0u;
+      if (tid == 0) s_kappa = -1;
+      __syncthreads();
+      double tot = 0.0, above = 0.0;
+      if (khi <= 0x7FFE) {
+        window_stream<1>(row, ua, ub, lane, rr, kk, klo, khi, wcnt, tot, above);
+      } else if (klo >= 0x8001) {
+        window_stream<2>(row, ua, ub, lane, rr, kk, klo, khi, wcnt, tot, above);
+      } else {
+        window_stream<0>(row, ua, ub, lane, rr, kk, klo, khi, wcnt, tot, above);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        tot += __shfl_xor_sync(0xffffffffu, tot, o);
+        above += __shfl_xor_sync(0xffffffffu, above, o);
+      }
+      if (lane == 0) {
+        s_red[wid] = tot;
+        s_red[kFastWarps + wid] = above;
+      }
+      __syncthreads();
+      tot = 0.0;
+      above = 0.0;
+      for (int q = 0; q < kFastWarps; ++q) {
+        tot += s_red[q];
+        above += s_red[kFastWarps + q];
+      }
+      target = a.top_p * tot;
+      const bool fin = isfinite(tot);
+      // the window's values from the top (thread t: keys khi - 4t ... khi - 4t - 3)
+      constexpr int KT = kWinKeys / kFastThreads;
+      double wm = 0.0;
+      float qk[KT];
+      unsigned ck[KT];
+#pragma unroll
+      for (int t = 0; t < KT; ++t) ck[t] = 0u;
+      const int top = khi - KT * tid;  // this thread's keys: top, top - 1, ..., top - KT + 1
+#pragma unroll
+      for (int t = 0; t < KT; ++t) {
+        const int key = top - t;
+        if (key >= klo) {
+          const int idx = key - klo;
+          unsigned sum = 0u;
+#pragma unroll
+          for (int v = 0; v < kFastWarps; ++v) sum += s_area[v * kWinKeys + idx];
+          ck[t] = sum;
+        }
+        qk[t] = ck[t] ? ex2((key16_value(static_cast<uint32_t>(key)) - rr) * kk) : 0.f;
+        wm += static_cast<double>(ck[t]) * static_cast<double>(qk[t]);
+      }
+      const double ex = block_scan<double, kFastThreads>(wm, s_dtmp);
+      if (fin && above < target) {
+        double run = above + ex;
+#pragma unroll
+        for (int t = 0; t < KT; ++t) {
+          const double mass = static_cast<double>(ck[t]) * static_cast<double>(qk[t]);
+          if (ck[t] && run < target && run + mass >= target) {
+            s_kappa = top - t;
+            s_before = run;
+            s_qk = static_cast<double>(qk[t]);
+            s_ck = ck[t];
+          }
+          run += mass;
+        }
+      }
+      __syncthreads();
+      if (!fin) {
+        hand = true;
+      } else if (s_kappa >= 0) {
+        done = true;
+      } else if (pass == 0) {  // the crossing lies above (below) the window: count the keys just above (below)
+        const bool up = !(above < target);
+        if (up ? khi >= kFiniteKeyHi : klo <= kFiniteKeyLo) {
+          hand = true;
+        } else if (tid == 0) {  // read by every thread after the barrier that opens the next pass
+          if (up) {
+            s_klo = khi + 1;
+            s_khi = min(khi + kWinKeys, kFiniteKeyHi);
+          } else {
+            s_khi = klo - 1;
+            s_klo = max(klo - kWinKeys, kFiniteKeyLo);
+          }
+        }
+      } else {
+        hand = true;
+      }
+      if (!done && !hand) __syncthreads();  // s_klo / s_khi written
+    }
+    // the reference r must lie close enough to the row's maximum that exp(-lf) stays a normal float for the
+    // sampling kernel
+    if (!done || s_before + static_cast<double>(s_ck) * s_qk > 1e26) {
+      if (tid == 0) a.flags[r] = 1;
+      __syncthreads();
+      continue;
+    }
+    const uint32_t kappa = key16_to_key32(static_cast<uint32_t>(s_kappa));
+    const double before = s_before, q = s_qk;
+    const unsigned c = s_ck;
+    double need = ceil((target - before) / q);
+    if (need < 1.0) need = 1.0;
+    const unsigned take = need < static_cast<double>(c) ? static_cast<unsigned>(need) : c;
+    const double kept = before + static_cast<double>(take) * q;
+    int64_t vcut = a.V - 1;
+    if (take < c) {  // the chunk that holds the take-th token at the cut value, then that token within it
+      if (tid == 0) {
+        const int idx = s_kappa - s_klo;
+        unsigned n = take;
+        int sel = kFastWarps - 1;
+        for (int v = 0; v < kFastWarps; ++v) {
+          const unsigned cv = s_area[v * kWinKeys + idx];
+          if (n <= cv) {
+            sel = v;
+            break;
+          }
+          n -= cv;
+        }
+        s_wsel = sel;
+        s_nth = n;
+      }
+      __syncthreads();
+      const int sa = min(Vu, s_wsel * cw), sb = min(Vu, sa + cw);
+      vcut = 8ll * sa + nth_equal<1, true, kFastWarps>(row + 16ll * sa, 8ll * (sb - sa), kappa, s_nth, s_wc, &s_v);
+    }
+    if (tid == 0) {
+      a.flags[r] = 0;
+      a.row_m[r] = rr;  // the reference of the masses: lf is relative to it
+      a.row_lf[r] = log(kept);
+      a.cut_key[r] = kappa;
+      a.cut_v[r] = static_cast<int32_t>(vcut);
+      if (tok >= 0) rs.xg[r] = s_xg;
+    }
+    __syncthreads();
+  }
+}
+
+cudaError_t launch_nucleus_fast(const NucleusArgs& a, cudaStream_t st) {
+  const size_t smem = static_cast<size_t>(2 * a.rs.B + 1) * sizeof(int);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t rows_max = static_cast<int64_t>(a.rs.B) * ((a.rs.K + 1) * a.rs.L + 1);
+  const dim3 grid(static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(rows_max, 4 * sms))));
+  if (smem > 48 * 1024) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(k_nucleus_fast, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  return launch_pdl(k_nucleus_fast, grid, dim3(kFastThreads), smem, st, a);
 }
 
 cudaError_t launch_nucleus(const NucleusArgs& a, int dtype, bool vec, cudaStream_t st) {

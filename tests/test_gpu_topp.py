@@ -262,3 +262,46 @@ def test_graph_replay_with_top_p_across_allocations():
         seen.add(tuple(rd["verify_len"]))
     assert len(seen) > 1
     assert ver_ws.status() & ~specv.DEV_NONFINITE == 0
+
+
+def _edge_rows_inputs(V, seed):
+    """Requests whose rows take every branch of the windowed nucleus kernel
+    (bf16 rows of 16-byte vectors, V >= 4096): constant rows (one tie value),
+    signed zeros, half the vocabulary at -inf, rows far below zero, a handful
+    of peaks a strided sample misses (the cut lies above the sampled window),
+    a very wide spread, and rows holding +inf or a NaN (handed to the exact
+    kernel, the request flagged)."""
+    x = synth.custom(B=9, L=3, V=V, K=2, T=1.0, dtype="bf16", n_peaks=0, draft_sigma=1.0, seed=seed, cid=700)
+    rng = np.random.default_rng(seed)
+    t = bf16_bits_to_f32(x.target).copy()
+    d = bf16_bits_to_f32(x.draft).copy()
+    t[0] = 0.0
+    d[0] = 1.0
+    t[1] = 0.0
+    t[1, :, ::3] = -0.0
+    d[1, :, :, 1::2] = -0.0
+    t[2, :, : V // 2] = -np.inf
+    d[2, :, :, V // 2:] = -np.inf
+    t[3] -= 50.0
+    d[3] -= 80.0
+    for i in range(t.shape[1]):  # four peaks between the sampled units
+        t[4, i, rng.choice(V, 4, replace=False) | 1] = 30.0
+    t[5] *= 8.0
+    d[5] *= 6.0
+    t[6, 1, 17] = np.inf
+    d[7, 1, 2, 5] = np.nan
+    t[8] = np.round(t[8] * 4) / 4  # few distinct values, many ties
+    x.target = synth.f32_to_bf16_bits(t)
+    x.draft = synth.f32_to_bf16_bits(d)
+    return x
+
+
+@pytest.mark.parametrize("top_p", [0.3, 0.9, 0.97])
+def test_windowed_nucleus_edge_rows(top_p):
+    x = _edge_rows_inputs(8192, seed=int(top_p * 100))
+    ref = _ref(x, top_p)
+    acc, out = _verify(to_torch(x), x, top_p)
+    acc, out = _cpu(acc), _cpu(out)
+    check_verify(acc, out, ref)
+    assert acc[6] == -1 and acc[7] == -1  # the non-finite rows flag their requests
+    assert (acc[[0, 1, 3, 4, 5, 8]] >= 0).all()
