@@ -22,7 +22,8 @@
 //     position (one barrier per round); the selected entries are then the
 //     first budget' - B positions;
 //     otherwise (larger windows, or a flagged score that may unsort a row) a
-//     radix select over the keys, 8-bit digits from the top, finds the cut:
+//     radix select over the keys, 8-bit digits from the highest bit on which
+//     two keys differ, finds the cut:
 //     per digit a 256-bin histogram of the entries that still match the
 //     prefix (one shared atomic per distinct digit of a warp, grouped with
 //     __match_any_sync) and one warp's suffix scan over it; the descent stops
@@ -87,6 +88,7 @@ __global__ void __launch_bounds__(kDvlThreads, 1) k_dvl_allocate(const float* __
   __shared__ int s_hist[256];
   __shared__ int s_tmp[kDvlWarps + 1];
   __shared__ int s_digit, s_k, s_binc, s_flag;
+  __shared__ unsigned long long s_or, s_and;
   pdl_wait();
   pdl_trigger();
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -94,7 +96,12 @@ __global__ void __launch_bounds__(kDvlThreads, 1) k_dvl_allocate(const float* __
   int* sRank = reinterpret_cast<int*>(sKey + n);  // index-order rank among the entries equal to the cut key
   int* lens = sRank + n;                           // verify_len + 1, then offsets
 
-  if (tid == 0) s_flag = 0;
+  if (tid == 0) {
+    s_flag = 0;
+    s_or = 0ull;
+    s_and = ~0ull;
+  }
+  for (int r = tid; r < B; r += kDvlThreads) lens[r] = 0;  // past the staged scores
   __syncthreads();
   int bad = 0;
   float* stage = reinterpret_cast<float*>(sKey + n);  // the scores, loaded coalesced (space reused below)
@@ -193,10 +200,34 @@ __global__ void __launch_bounds__(kDvlThreads, 1) k_dvl_allocate(const float* __
   unsigned long long prefix = ~0ull, mask = ~0ull;
   int k = 0, binc = 0;
   if (take > 0) {
-    prefix = 0ull;
-    mask = 0ull;
+    // the bits above the highest one on which two keys differ are common to all: the descent starts below
+    // them (products in [0, 1] share the sign and most exponent bits, a whole digit or more)
+    unsigned long long o = 0ull, a = ~0ull;
+    for (int e = tid; e < n; e += kDvlThreads) {
+      o |= sKey[e];
+      a &= sKey[e];
+    }
+    const unsigned ohi = __reduce_or_sync(0xffffffffu, static_cast<unsigned>(o >> 32));
+    const unsigned olo = __reduce_or_sync(0xffffffffu, static_cast<unsigned>(o));
+    const unsigned ahi = __reduce_and_sync(0xffffffffu, static_cast<unsigned>(a >> 32));
+    const unsigned alo = __reduce_and_sync(0xffffffffu, static_cast<unsigned>(a));
+    if (lane == 0) {
+      atomicOr(&s_or, (static_cast<unsigned long long>(ohi) << 32) | olo);
+      atomicAnd(&s_and, (static_cast<unsigned long long>(ahi) << 32) | alo);
+    }
+    __syncthreads();
+    const unsigned long long diff = s_or ^ s_and;
     k = take;  // rank (1-based, descending) of the wanted entry among those matching the prefix
-    for (int shift = 56; shift >= 0; shift -= 8) {
+    if (diff == 0ull) {  // one key: the cut is that key, taken by flat index
+      prefix = s_and;
+      binc = n;
+    } else {
+      const int hb = 63 - __clzll(static_cast<long long>(diff));
+      mask = hb == 63 ? 0ull : ~((2ull << hb) - 1ull);
+      prefix = s_and & mask;
+    }
+    for (int shift = max(0, (diff == 0ull ? 0 : 63 - __clzll(static_cast<long long>(diff))) - 7);
+         diff != 0ull; shift = max(0, shift - 8)) {
       if (tid < 256) s_hist[tid] = 0;
       __syncthreads();
       for (int base = wid * 32; base < n; base += kDvlThreads) {  // warp-uniform trips: full-warp intrinsics
@@ -240,7 +271,7 @@ __global__ void __launch_bounds__(kDvlThreads, 1) k_dvl_allocate(const float* __
       mask |= 255ull << shift;
       k = s_k;
       binc = s_binc;
-      if (binc == k) break;  // the whole bin is taken: nothing below this digit matters (block-uniform)
+      if (binc == k || shift == 0) break;  // the whole bin is taken, or every bit decided (block-uniform)
     }
   }
 
@@ -251,14 +282,15 @@ __global__ void __launch_bounds__(kDvlThreads, 1) k_dvl_allocate(const float* __
     __syncthreads();
     block_exclusive_scan<kDvlThreads>(sRank, n, s_tmp);
   }
-  // verify_len[b]: selected entries of row b (a prefix of the row when every score is in [0, 1])
+  // verify_len[b]: selected entries of row b (a prefix of the row when every score is in [0, 1]), one thread
+  // per entry
+  for (int e = tid; e < n; e += kDvlThreads) {
+    const unsigned long long um = sKey[e] & mask;
+    if (um > prefix || (um == prefix && take > 0 && (rank_eq ? sRank[e] < k : true))) atomicAdd(&lens[e / L], 1);
+  }
+  __syncthreads();
   for (int r = tid; r < B; r += kDvlThreads) {
-    int ell = 0;
-    for (int i = 0; i < L; ++i) {
-      const int e = r * L + i;
-      const unsigned long long um = sKey[e] & mask;
-      ell += (um > prefix || (um == prefix && take > 0 && (rank_eq ? sRank[e] < k : true))) ? 1 : 0;
-    }
+    const int ell = lens[r];
     verify_len[r] = ell;
     lens[r] = ell + 1;
   }
