@@ -102,18 +102,59 @@ __global__ void __launch_bounds__(kDvlThreads, 1) k_dvl_allocate(const float* __
     s_and = ~0ull;
   }
   for (int r = tid; r < B; r += kDvlThreads) lens[r] = 0;  // past the staged scores
-  __syncthreads();
   int bad = 0;
-  float* stage = reinterpret_cast<float*>(sKey + n);  // the scores, loaded coalesced (space reused below)
-  for (int e = tid; e < n; e += kDvlThreads) stage[e] = scores[e];
-  __syncthreads();
-  for (int r = tid; r < B; r += kDvlThreads) {
-    double P = 1.0;
-    for (int i = 0; i < L; ++i) {
-      const float sv = stage[r * L + i];
-      bad |= !(sv >= 0.f && sv <= 1.f);
-      P = P * static_cast<double>(sv);
-      sKey[r * L + i] = p_key(P);
+  unsigned long long kor = 0ull, kand = ~0ull;  // OR and AND of this thread's keys (the radix descent's start)
+  if (L % 4 == 0 && L <= kDvlMaxL && (reinterpret_cast<uintptr_t>(scores) & 15) == 0) {
+    // a thread's row as 16-byte vectors straight into registers (one memory round trip), then the products
+    __syncthreads();  // s_or / s_and initialised
+    for (int r = tid; r < B; r += kDvlThreads) {
+      float4 v[kDvlMaxL / 4];
+#pragma unroll
+      for (int q = 0; q < kDvlMaxL / 4; ++q)
+        if (q < L / 4) v[q] = __ldg(reinterpret_cast<const float4*>(scores + static_cast<int64_t>(r) * L) + q);
+      double P = 1.0;
+#pragma unroll
+      for (int q = 0; q < kDvlMaxL / 4; ++q) {
+        if (q < L / 4) {
+          const float sv[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            bad |= !(sv[c] >= 0.f && sv[c] <= 1.f);
+            P = P * static_cast<double>(sv[c]);
+            const unsigned long long key = p_key(P);
+            sKey[r * L + 4 * q + c] = key;
+            kor |= key;
+            kand &= key;
+          }
+        }
+      }
+    }
+  } else {
+    __syncthreads();  // s_or / s_and initialised
+    float* stage = reinterpret_cast<float*>(sKey + n);  // the scores, loaded coalesced (space reused below)
+    for (int e = tid; e < n; e += kDvlThreads) stage[e] = scores[e];
+    __syncthreads();
+    for (int r = tid; r < B; r += kDvlThreads) {
+      double P = 1.0;
+      for (int i = 0; i < L; ++i) {
+        const float sv = stage[r * L + i];
+        bad |= !(sv >= 0.f && sv <= 1.f);
+        P = P * static_cast<double>(sv);
+        const unsigned long long key = p_key(P);
+        sKey[r * L + i] = key;
+        kor |= key;
+        kand &= key;
+      }
+    }
+  }
+  {  // the bits above the highest one on which two keys differ are common to all (used by the radix descent)
+    const unsigned ohi = __reduce_or_sync(0xffffffffu, static_cast<unsigned>(kor >> 32));
+    const unsigned olo = __reduce_or_sync(0xffffffffu, static_cast<unsigned>(kor));
+    const unsigned ahi = __reduce_and_sync(0xffffffffu, static_cast<unsigned>(kand >> 32));
+    const unsigned alo = __reduce_and_sync(0xffffffffu, static_cast<unsigned>(kand));
+    if (lane == 0) {
+      atomicOr(&s_or, (static_cast<unsigned long long>(ohi) << 32) | olo);
+      atomicAnd(&s_and, (static_cast<unsigned long long>(ahi) << 32) | alo);
     }
   }
   if (bad) atomicOr(&s_flag, kFlagScores);
@@ -202,20 +243,6 @@ __global__ void __launch_bounds__(kDvlThreads, 1) k_dvl_allocate(const float* __
   if (take > 0) {
     // the bits above the highest one on which two keys differ are common to all: the descent starts below
     // them (products in [0, 1] share the sign and most exponent bits, a whole digit or more)
-    unsigned long long o = 0ull, a = ~0ull;
-    for (int e = tid; e < n; e += kDvlThreads) {
-      o |= sKey[e];
-      a &= sKey[e];
-    }
-    const unsigned ohi = __reduce_or_sync(0xffffffffu, static_cast<unsigned>(o >> 32));
-    const unsigned olo = __reduce_or_sync(0xffffffffu, static_cast<unsigned>(o));
-    const unsigned ahi = __reduce_and_sync(0xffffffffu, static_cast<unsigned>(a >> 32));
-    const unsigned alo = __reduce_and_sync(0xffffffffu, static_cast<unsigned>(a));
-    if (lane == 0) {
-      atomicOr(&s_or, (static_cast<unsigned long long>(ohi) << 32) | olo);
-      atomicAnd(&s_and, (static_cast<unsigned long long>(ahi) << 32) | alo);
-    }
-    __syncthreads();
     const unsigned long long diff = s_or ^ s_and;
     k = take;  // rank (1-based, descending) of the wanted entry among those matching the prefix
     if (diff == 0ull) {  // one key: the cut is that key, taken by flat index
