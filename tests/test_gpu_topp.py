@@ -305,3 +305,16 @@ def test_windowed_nucleus_edge_rows(top_p):
     check_verify(acc, out, ref)
     assert acc[6] == -1 and acc[7] == -1  # the non-finite rows flag their requests
     assert (acc[[0, 1, 3, 4, 5, 8]] >= 0).all()
+
+
+@pytest.mark.parametrize("dtype,V", [("f32", 32768), ("bf16", 20001)])
+def test_exact_nucleus_kernel_rows(dtype, V):
+    """Rows the windowed kernel does not take (fp32 rows; bf16 rows whose
+    length is not a whole number of 16-byte vectors) go to the exact kernel
+    alone: its fp32 radix descent and its scalar bf16 path, at sizes that span
+    many digits and a ragged tail."""
+    x = redraw_from_filtered(synth.custom(B=6, L=8, V=V, K=2, T=1.2, dtype=dtype, n_peaks=6, peak=5.0,
+                                          draft_sigma=1.0, seed=V % 97, cid=710 + (dtype == "f32")), 0.9, seed=41)
+    ref = _ref(x, 0.9)
+    acc, out = _verify(to_torch(x), x, 0.9)
+    check_verify(_cpu(acc), _cpu(out), ref)
