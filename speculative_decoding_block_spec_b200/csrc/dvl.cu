@@ -25,8 +25,9 @@
 //     radix select over the keys, 8-bit digits from the highest bit on which
 //     two keys differ, finds the cut:
 //     per digit a 256-bin histogram of the entries that still match the
-//     prefix (one shared atomic per distinct digit of a warp, grouped with
-//     __match_any_sync) and one warp's suffix scan over it; the descent stops
+//     prefix (one shared atomic per entry; starting below the common bits
+//     spreads the first digit over many bins) and one warp's suffix scan over
+//     it; the descent stops
 //     at the first digit whose bin is taken whole; entries above the cut are
 //     selected, and of those equal to it the first ones by flat index;
 //  3. verify_len[b] = selected entries of row b; an exclusive scan of
@@ -257,12 +258,11 @@ __global__ void __launch_bounds__(kDvlThreads, 1) k_dvl_allocate(const float* __
          diff != 0ull; shift = max(0, shift - 8)) {
       if (tid < 256) s_hist[tid] = 0;
       __syncthreads();
-      for (int base = wid * 32; base < n; base += kDvlThreads) {  // warp-uniform trips: full-warp intrinsics
+      for (int base = wid * 32; base < n; base += kDvlThreads) {
         const int e = base + lane;
         const unsigned long long u = e < n ? sKey[e] : 0ull;
         const int d = (e < n && (u & mask) == prefix) ? static_cast<int>((u >> shift) & 255) : 256;
-        const unsigned peers = __match_any_sync(0xffffffffu, d);  // one atomic per distinct digit of the warp
-        if (d < 256 && lane == __ffs(peers) - 1) atomicAdd(&s_hist[d], __popc(peers));
+        if (d < 256) atomicAdd(&s_hist[d], 1);
       }
       __syncthreads();
       if (wid == 0) {  // lane l owns digits 255 - 8l ... 248 - 8l (descending)
