@@ -15,21 +15,14 @@
 //  1. one thread per request forms its products in fp64, left to right, and
 //     stores them as 64-bit keys whose unsigned order is the order of P
 //     (+0 and -0 are one key, as they compare equal);
-//  2. with every score in [0, 1] each row is already sorted in the global
-//     order (P desc, flat index asc), so for B <= 32 and B*L <= 4096 the B rows are
-//     merged bottom-up: in each of ceil(log2 B) rounds every entry finds its
-//     rank in the partner list by binary search and moves to its merged
-//     position (one barrier per round); the selected entries are then the
-//     first budget' - B positions;
-//     otherwise (larger windows, or a flagged score that may unsort a row) a
-//     radix select over the keys, 8-bit digits from the highest bit on which
-//     two keys differ, finds the cut:
-//     per digit a 256-bin histogram of the entries that still match the
-//     prefix (one shared atomic per entry; starting below the common bits
-//     spreads the first digit over many bins) and one warp's suffix scan over
-//     it; the descent stops
-//     at the first digit whose bin is taken whole; entries above the cut are
-//     selected, and of those equal to it the first ones by flat index;
+//  2. a radix select over the keys, 8-bit digits from the highest bit on
+//     which two keys differ, finds the cut: per digit a 256-bin histogram of
+//     the entries that still match the prefix (one shared atomic per entry;
+//     starting below the common bits spreads the first digit over many bins)
+//     and one warp's suffix scan over it; the descent stops at the first digit
+//     whose bin is taken whole; entries above the cut are selected, and of
+//     those equal to it the first ones by flat index (a block scan of the
+//     equal entries' flags);
 //  3. verify_len[b] = selected entries of row b; an exclusive scan of
 //     verify_len + 1 gives the offsets, from which the slot map is filled.
 // k_dvl_pack then copies the selected dense target rows into the
@@ -47,10 +40,6 @@ namespace specv {
 constexpr int kDvlThreads = SPECV_DVL_THREADS;  // one block; 256 ... 1024 threads
 constexpr int kDvlWarps = kDvlThreads / 32;
 constexpr int kDvlMaxL = 32;  // SPEC_MAX_L
-constexpr int kDvlMergeMax = 4096;  // B*L merged in shared memory (two key / index buffers)
-// Merge rounds grow with log2 B while the radix select takes about four digits whatever B: measured per launch
-// on B200 (L = 16), merge 4.9 / 7.4 / 9.9 us and radix 6.2 / 7.4 / 8.2 us at B = 8 / 32 / 64.
-constexpr int kDvlMergeMaxB = 32;
 
 // Order-preserving key of a product: unsigned order of the key = numeric
 // order of P (negative values below +0; -0 maps to the key of +0; a NaN,
@@ -163,79 +152,6 @@ __global__ void __launch_bounds__(kDvlThreads, 1) k_dvl_allocate(const float* __
 
   const int64_t cap = static_cast<int64_t>(B) * (L + 1);
   const int take = static_cast<int>(std::min<int64_t>(budget, cap)) - B;  // 0 <= take <= n
-  if (n <= kDvlMergeMax && B <= kDvlMergeMaxB && s_flag == 0) {  // block-uniform: every row sorted, merge them
-    unsigned long long* kA = sKey;
-    unsigned long long* kB = sKey + n;
-    uint32_t* iA = reinterpret_cast<uint32_t*>(sKey + 2 * n);
-    uint32_t* iB = iA + n;
-    uint32_t* hA = iB + n;  // the keys' top 32 bits: most comparisons end there (half the shared traffic)
-    uint32_t* hB = hA + n;
-    int* cnt = reinterpret_cast<int*>(hB + n);  // [B + 1]: selected entries per row, then lengths / offsets
-    for (int e = tid; e < n; e += kDvlThreads) {
-      iA[e] = static_cast<uint32_t>(e);
-      hA[e] = static_cast<uint32_t>(kA[e] >> 32);
-    }
-    for (int r = tid; r <= B; r += kDvlThreads) cnt[r] = 0;
-    __syncthreads();
-    for (int W = L; W < n; W *= 2) {  // lists of W entries, merged in pairs
-      for (int e = tid; e < n; e += kDvlThreads) {
-        const int base = (e / (2 * W)) * (2 * W);
-        const int mid = min(base + W, n), end = min(base + 2 * W, n);
-        const unsigned long long ke = kA[e];
-        const uint32_t ie = iA[e], he = hA[e];
-        // entries of the other list that precede (ke, ie) in the order (key desc, index asc) form a prefix
-        int lo = e < mid ? mid : base, hi = e < mid ? end : mid;
-        const int first = lo;
-        while (lo < hi) {
-          const int md = (lo + hi) >> 1;
-          const uint32_t hm = hA[md];
-          bool before = hm > he;
-          if (hm == he) {  // equal top halves: the full keys, then the flat index
-            const unsigned long long km = kA[md];
-            before = km > ke || (km == ke && iA[md] < ie);
-          }
-          if (before) lo = md + 1; else hi = md;
-        }
-        const int pos = base + (e < mid ? e - base : e - mid) + (lo - first);
-        kB[pos] = ke;
-        iB[pos] = ie;
-        hB[pos] = he;
-      }
-      __syncthreads();
-      unsigned long long* tk = kA; kA = kB; kB = tk;
-      uint32_t* ti = iA; iA = iB; iB = ti;
-      ti = hA; hA = hB; hB = ti;
-    }
-    for (int q = tid; q < take; q += kDvlThreads) atomicAdd(&cnt[iA[q] / L], 1);  // the first take are selected
-    __syncthreads();
-    for (int r = tid; r < B; r += kDvlThreads) {
-      const int ell = cnt[r];
-      verify_len[r] = ell;
-      cnt[r] = ell + 1;
-    }
-    __syncthreads();
-    if (wid == 0) {  // exclusive scan of the lengths + 1 by one warp: lane l owns a contiguous run
-      const int per = (B + 31) / 32, lo = min(B, lane * per), hi = min(B, lo + per);
-      int run = 0;
-      for (int r = lo; r < hi; ++r) run += cnt[r];
-      int incl = run;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-      }
-      int acc = incl - run;
-      for (int r = lo; r < hi; ++r) {
-        const int t = cnt[r];
-        cnt[r] = acc;
-        acc += t;
-      }
-      if (lane == 31) cnt[B] = incl;
-    }
-    __syncthreads();
-    write_offsets_and_slots(cnt, B, L, budget, cnt[B], offsets, slot_map);
-    return;  // scores all in [0, 1]: no flag to raise
-  }
   // The cut: entries whose key, under `mask`, is above `prefix` are selected; of those equal to it under the
   // mask, all are selected when the bin holds exactly the k still wanted, else (equal full keys) the first k
   // by flat index. take == 0 selects nothing: no masked key exceeds the all-ones prefix.
@@ -368,13 +284,9 @@ __global__ void __launch_bounds__(kThreads) k_dvl_pack(const char* __restrict__ 
 cudaError_t launch_dvl(const float* scores, int B, int L, int budget, int32_t* verify_len, int32_t* offsets,
                        int32_t* slot_map, int* status, cudaStream_t st) {
   const int64_t n = static_cast<int64_t>(B) * L;
-  // radix path: keys + equal ranks + lengths; merge path (B <= kDvlMergeMaxB, B*L <= kDvlMergeMax): two key,
-  // index and key-prefix buffers
-  const size_t radix = static_cast<size_t>(n) * (sizeof(unsigned long long) + sizeof(int)) +
-                       static_cast<size_t>(B + 1) * sizeof(int);
-  const size_t merge = static_cast<size_t>(n) * 2 * (sizeof(unsigned long long) + 2 * sizeof(uint32_t)) +
-                       static_cast<size_t>(B + 1) * sizeof(int);
-  const size_t smem = (n <= kDvlMergeMax && B <= kDvlMergeMaxB) ? std::max(radix, merge) : radix;
+  // keys, equal-key ranks, lengths
+  const size_t smem = static_cast<size_t>(n) * (sizeof(unsigned long long) + sizeof(int)) +
+                      static_cast<size_t>(B + 1) * sizeof(int);
   if (smem > 48 * 1024) {
     const cudaError_t e =
         cudaFuncSetAttribute(k_dvl_allocate, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
