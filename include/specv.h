@@ -223,11 +223,16 @@ int spec_verify_mixture(const void* target_logits, const int32_t* target_row_off
  *              once (it also serves the unfiltered calls of the same shape).
  * Other arguments and limits as spec_verify_block / spec_verify_mixture
  * (K = 1 and w = 1 for the block variant).
- * Execution: three launches chained with programmatic dependent launch:
- * the statistics of the verify window plus each request's bonus row; a
- * nucleus kernel that finds each row's cut (a radix descent over the
- * logits' order keys with exact fixed-point masses, then the tie cut by
- * token index); the accept / sample stage with the filtered rows.
+ * Execution: launches chained with programmatic dependent launch, over the
+ * verify window plus each request's bonus row. For bf16 rows of 16-byte
+ * vectors with V >= 4096 a windowed nucleus kernel finds each row's
+ * normaliser and cut from one pass (the keys near the cut, chosen from a
+ * strided sample, counted per value; every token's mass summed); the exact
+ * nucleus kernel then takes only the rows it hands over (a NaN or an
+ * infinity, or a crossing outside its window twice). Other rows go to the
+ * exact kernel alone (bf16 value counts, or for fp32 a radix descent over
+ * the logits' order keys with exact fixed-point masses, then the tie cut by
+ * token index). The accept / sample stage follows with the filtered rows.
  */
 size_t spec_verify_top_p_workspace_size(int B, int L, int K, int64_t V);
 
