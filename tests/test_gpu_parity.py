@@ -447,6 +447,25 @@ def test_dvl_ties_zeros_and_unsorted_rows(case):
         np.testing.assert_array_equal(_cpu(sm), ref["slot_map"])
 
 
+def test_dvl_misaligned_scores_take_the_staged_load():
+    """Scores whose rows are not 16-byte aligned (a view 4 bytes into an
+    allocation) are staged through shared memory instead of loaded as
+    vectors; the allocation is the same."""
+    rng = np.random.default_rng(11)
+    B, L = 64, 16
+    s = -np.sort(-rng.beta(6.0, 2.0, size=(B, L)), axis=1).astype(np.float32)
+    flat = torch.zeros(B * L + 1, dtype=torch.float32, device="cuda")
+    flat[1:] = torch.from_numpy(s.reshape(-1)).cuda()
+    view = flat[1:].view(B, L)
+    assert view.data_ptr() % 16 != 0
+    for budget in (B, B * (L + 1) // 2, B * (L + 1)):
+        ref = oracle.dvl_allocate(s, budget)
+        vl, off, sm = specv.dvl_allocate_pack(view, budget)
+        np.testing.assert_array_equal(_cpu(vl), ref["verify_len"])
+        np.testing.assert_array_equal(_cpu(off), ref["offsets"])
+        np.testing.assert_array_equal(_cpu(sm), ref["slot_map"])
+
+
 def test_dvl_flags_bad_scores():
     s = torch.full((4, 4), 0.5, device="cuda")
     s[2, 1] = 1.5
